@@ -1,0 +1,371 @@
+"""Benchmark of the Sol-Attn forward on B200.
+
+One step = one full forward (block pooling, moments + thresholds, fused
+routing / exact / approximation kernel) over the Wan-2.1-14B-like
+self-attention shape: B=1, H=40, L=75,600 (21x45x80 latent grid), d=128,
+64-token blocks (ragged 16-token tail), C=64, beta=1.0, synthetic seeded
+Fourier-feature inputs.  The same shape in the kernel's own select-all
+(dense) mode gives the speedup.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun (N > 1) every rank runs its own batch element of the same
+shape (weak scaling, no data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sol_attn fwd ms & executed TFLOPS (% BF16 peak); speedup vs own dense mode"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic():
+    """dram bytes per fused-kernel launch from the committed ncu summary, if that
+    summary was taken on the current kernel source (else None)."""
+    import hashlib
+    summ = os.path.join(ROOT, "profiles", "fused_kernel_traffic.txt")
+    src = os.path.join(ROOT, "block_sparse_attention_moments_b200", "csrc", "fused.cuh")
+    if not os.path.exists(summ):
+        return None
+    fields = {}
+    with open(summ) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                key, val = line.split(":", 1)
+                fields[key.strip()] = val.strip()
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    if fields.get("fused_cuh_sha256") != h or "dram_bytes_per_launch_full" not in fields:
+        return None
+    return float(fields["dram_bytes_per_launch_full"])
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sol_attn_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.dev)], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    torch.cuda.set_device(local)
+    return rank, world, local, pg
+
+
+def max_over_ranks(x: float, pg) -> float:
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, pg) -> float:
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_inputs(wl, rank: int):
+    """bf16 bits of this rank's batch element: heads b*H .. b*H+H-1 of a batch of world size."""
+    import dataclasses
+
+    from synth import fourier_inputs
+    big = dataclasses.replace(wl, B=rank + 1)
+    heads = list(range(rank * wl.H, (rank + 1) * wl.H))
+    q, k, v = fourier_inputs(big, heads=heads)
+    return q[rank:rank + 1], k[rank:rank + 1], v[rank:rank + 1]
+
+
+def cpu_baseline(wl, beta: float, budget_rows: int):
+    """The fp64 oracle, as it stands, on a bounded sample: one head, `budget_rows`
+    query blocks spread over the sequence (plus that head's pooling and moments)."""
+    import numpy as np
+
+    from oracle import sol_attn_head
+    from synth import bf16_bits_to_f64, fourier_inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count() or 1
+    q, k, v = fourier_inputs(wl, heads=[0])
+    q, k, v = (bf16_bits_to_f64(x[0, 0]) for x in (q, k, v))
+    rows = sorted(set(np.linspace(0, wl.N - 1, budget_rows).astype(int).tolist()))
+    t0 = time.perf_counter()
+    r = sol_attn_head(q, k, v, beta, rows=rows)
+    dt = time.perf_counter() - t0
+    d, N = wl.d, wl.N
+    approx = not math.isinf(beta)
+    flops = sum(4.0 * 64 * 64 * d * int(r["counts"][i]) + (4.0 * 64 * d * N if approx else 0) + 2.0 * d * N
+                for i in rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": int(cores), "kind": "oracle",
+            "sample": f"1 of {wl.B * wl.H} heads, {len(rows)} of {N} query blocks (fp64 numpy, incl. that head's "
+                      f"pooling and moments), {dt:.1f} s", "seconds": dt, "flops": flops}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle timed on the host cores (rank 0 only)."""
+    from synth import WORKLOADS
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        cpu_baseline(wl, args.beta, 4)
+    vals, secs, flops = [], 0.0, 0.0
+    cb = None
+    for _ in range(args.steps):
+        cb = cpu_baseline(wl, args.beta, args.ref_rows)
+        secs += cb["seconds"]
+        flops += cb["flops"]
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} L={wl.L} d={wl.d} block=64 C={wl.chunk} beta={args.beta}",
+                   "sample_per_step": cb["sample"] if cb else None},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cb["cores"] if cb else None, "kind": "oracle",
+                         "sample": cb["sample"] if cb else None},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="wan")
+    ap.add_argument("--beta", type=float, default=1.0)
+    ap.add_argument("--ref-rows", type=int, default=48, help="query blocks per reference step")
+    ap.add_argument("--cpu-rows", type=int, default=768, help="query blocks in the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_moments_b200 as sa
+    from synth import WORKLOADS
+
+    rank, world, local, pg = dist_setup(args.gpus)
+    wl = WORKLOADS[args.workload]
+    B, H, L, d, C = 1, wl.H, wl.L, wl.d, wl.chunk
+    N = wl.N
+    qb, kb, vb = rank_inputs(wl, rank)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = dev(qb), dev(kb), dev(vb)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def step(beta, flags, ev=None):
+        if ev is None:
+            sa.stage_pool(q, k, v, stream=stream)
+            sa.stage_threshold(B, H, L, d, beta, flags=flags, stream=stream)
+            sa.stage_fused(q, k, v, out, C, flags=flags, stream=stream)
+            return
+        ev[0].record(stream)
+        sa.stage_pool(q, k, v, stream=stream)
+        ev[1].record(stream)
+        sa.stage_threshold(B, H, L, d, beta, flags=flags, stream=stream)
+        ev[2].record(stream)
+        sa.stage_fused(q, k, v, out, C, flags=flags, stream=stream)
+        ev[3].record(stream)
+
+    def timed(beta, flags, sampler=None):
+        for _ in range(args.warmup):
+            step(beta, flags)
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+        if sampler:
+            sampler.start()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for s in range(args.steps):
+            step(beta, flags, evs[s])
+        end.record(stream)
+        torch.cuda.synchronize()
+        clocks = sampler.stop() if sampler else None
+        if pg is not None:
+            pg.barrier()
+        total_ms = start.elapsed_time(end)
+        per = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(3)]
+        counts = sa.stats(B, H, L, stream=stream)
+        torch.cuda.synchronize()
+        pairs = int(counts.to(torch.int64).sum().item())
+        return total_ms, per, pairs, clocks
+
+    # sparse run (the headline) and the same kernel in select-all (dense) mode
+    sampler = ClockSampler(local)
+    total_ms, per_ms, pairs, clocks = timed(args.beta, 0, sampler)
+    dense_ms, dense_per, dense_pairs, _ = timed(-math.inf, sa.FLAG_SELECT_ALL)
+    flops_step = sa.executed_flops(pairs, B, H, L, d, approx=True)
+    fused_flops = flops_step  # the fused kernel executes all exact, proxy and routing FLOPs
+    step_ms = max_over_ranks(total_ms / args.steps, pg)
+    fused_ms = max_over_ranks(per_ms[2], pg)
+    all_flops = sum_over_ranks(flops_step, pg)
+    dense_step_ms = max_over_ranks(dense_ms / args.steps, pg)
+    value = all_flops / (step_ms * 1e-3) / 1e12
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.from_numpy(qb.view(np.int16)).pin_memory()
+        hk = torch.from_numpy(kb.view(np.int16)).pin_memory()
+        hv = torch.from_numpy(vb.view(np.int16)).pin_memory()
+        ho = torch.empty_like(hq).pin_memory()
+        for _ in range(2):
+            sa.forward_host(hq, hk, hv, args.beta, C, out=ho)
+        if pg is not None:
+            pg.barrier()
+        ksteps = max(2, min(args.steps, 5))
+        t0 = time.perf_counter()
+        for _ in range(ksteps):
+            sa.forward_host(hq, hk, hv, args.beta, C, out=ho)
+        e2e_s = max_over_ranks((time.perf_counter() - t0) / ksteps, pg)
+        nbytes = q.numel() * 2
+        e2e = {"value": all_flops / e2e_s / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": 3 * nbytes,
+               "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_s * 1e3}
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved = fused_flops / (fused_ms * 1e-3) / 1e12
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cb = cpu_baseline(wl, args.beta, args.cpu_rows)
+        cpu = {k2: cb[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name}: Wan-2.1-14B-like self-attention B=1 H={H} L={L} (21x45x80) d={d} "
+                               f"block=64 C={C} beta={args.beta}, bf16 Fourier-feature Q/K, Gaussian V",
+                   "per_gpu_batch": 1, "global_batch": world, "seq_len": L, "parallelism": f"dp{world} (weak)",
+                   "l2": "inputs (2.3 GB/step) larger than L2 (126 MB)"},
+        "ms_per_call": step_ms,
+        "pct_bf16_peak": 100.0 * value / world / peak,
+        "stage_ms": {"pool": per_ms[0], "threshold": per_ms[1], "fused": per_ms[2]},
+        "density": pairs / (B * H * N * N),
+        "dense_ms_per_call": dense_step_ms,
+        "dense_tflops": sa.executed_flops(dense_pairs, B, H, L, d, approx=False) / (dense_step_ms * 1e-3) / 1e12,
+        "speedup_vs_dense": dense_step_ms / step_ms,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": load_traffic(),
+                     "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"
+                     else "fallback 1.59 PFLOP/s", "frac_of_sustained": achieved / peak_sus,
+                     "kernel": "sol_attn_fused_kernel", "algorithmic_flops_per_launch": fused_flops},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * sa.kernels_per_forward(),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

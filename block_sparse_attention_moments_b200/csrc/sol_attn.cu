@@ -1,0 +1,534 @@
+// sol_attn.cu — C ABI of the Sol-Attn forward (declared in include/sol_attn.h):
+// argument checks, the per-device workspace, TMA descriptor set-up and the
+// launches of the three kernels (pool, moments + thresholds, fused attention).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "fused.cuh"
+#include "moments.cuh"
+#include "pool.cuh"
+#include "sol_attn.h"
+
+using namespace solattn;
+
+namespace {
+
+constexpr int kBlock = 64;
+constexpr int kMaxL = 1 << 20;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // bounded device waits: 2 s
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                        \
+  do {                                                                                        \
+    cudaError_t e_ = (expr);                                                                  \
+    if (e_ != cudaSuccess) return fail(SOL_ATTN_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+// ------------------------------------------------------------------ workspace
+struct Shape {
+  int B = 0, H = 0, L = 0, d = 0;
+  bool operator==(const Shape& o) const { return B == o.B && H == o.H && L == o.L && d == o.d; }
+};
+
+struct Workspace {
+  void* base = nullptr;
+  size_t bytes = 0;
+  // carved views
+  float* qbar = nullptr;
+  float* kbar = nullptr;
+  __nv_bfloat16* kbar_bf = nullptr;
+  __nv_bfloat16* kbar_lo = nullptr;
+  __nv_bfloat16* vhat_bf = nullptr;
+  double* mom_mean = nullptr;
+  double* mom_cov = nullptr;
+  float* tau = nullptr;
+  int* counts = nullptr;
+  unsigned* counter = nullptr;   // fixed 256-byte block, allocated once per device:
+  unsigned* status = nullptr;    // [0] work counter, [32] sticky status word
+  void* ctl_block = nullptr;
+  Shape shape;        // shape the views are carved for
+  int stage = 0;      // 0 none, 1 pooled, 2 thresholds, 3 fused done
+  Shape last_fused;   // shape of the last completed forward (for stats)
+  // host-buffer entry point staging
+  void* host_stage = nullptr;
+  size_t host_stage_bytes = 0;
+  cudaStream_t host_stream = nullptr;
+};
+
+constexpr int kMaxDevices = 64;
+Workspace g_ws[kMaxDevices];
+std::mutex g_mu;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t layout(const Shape& s, Workspace* w, char* base) {
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const size_t N = (static_cast<size_t>(s.L) + kBlock - 1) / kBlock;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return base ? base + o : nullptr;
+  };
+  char* p_qbar = take(BH * N * s.d * 4);
+  char* p_kbar = take(BH * N * s.d * 4);
+  char* p_kbf = take(BH * N * s.d * 2);
+  char* p_klo = take(BH * N * s.d * 2);
+  char* p_vbf = take(BH * N * s.d * 2);
+  char* p_mean = take(BH * s.d * 8);
+  char* p_cov = take(BH * s.d * s.d * 8);
+  char* p_tau = take(BH * N * 4);
+  char* p_cnt = take(BH * N * 4);
+  if (w && base) {
+    w->qbar = reinterpret_cast<float*>(p_qbar);
+    w->kbar = reinterpret_cast<float*>(p_kbar);
+    w->kbar_bf = reinterpret_cast<__nv_bfloat16*>(p_kbf);
+    w->kbar_lo = reinterpret_cast<__nv_bfloat16*>(p_klo);
+    w->vhat_bf = reinterpret_cast<__nv_bfloat16*>(p_vbf);
+    w->mom_mean = reinterpret_cast<double*>(p_mean);
+    w->mom_cov = reinterpret_cast<double*>(p_cov);
+    w->tau = reinterpret_cast<float*>(p_tau);
+    w->counts = reinterpret_cast<int*>(p_cnt);
+  }
+  return off;
+}
+
+int current_device(int* dev) {
+  CUDA_TRY(cudaGetDevice(dev));
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(SOL_ATTN_ERR_UNSUPPORTED, "device index %d too large", *dev);
+  return SOL_ATTN_OK;
+}
+
+int check_arch(int dev) {
+  static int checked[kMaxDevices] = {0};
+  if (checked[dev] == 1) return SOL_ATTN_OK;
+  int major = 0, minor = 0;
+  CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0)
+    return fail(SOL_ATTN_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev, major,
+                minor);
+  checked[dev] = 1;
+  return SOL_ATTN_OK;
+}
+
+// Make the workspace of the current device fit shape s (grow-only allocation).
+int ensure_ws(const Shape& s, Workspace** out) {
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  if ((rc = check_arch(dev))) return rc;
+  Workspace& w = g_ws[dev];
+  if (!w.ctl_block) {
+    CUDA_TRY(cudaMalloc(&w.ctl_block, 256));
+    CUDA_TRY(cudaMemset(w.ctl_block, 0, 256));
+    w.counter = static_cast<unsigned*>(w.ctl_block);
+    w.status = static_cast<unsigned*>(w.ctl_block) + 32;
+  }
+  const size_t need = layout(s, nullptr, nullptr);
+  if (need > w.bytes) {
+    if (w.base) CUDA_TRY(cudaFree(w.base));
+    w.base = nullptr;
+    w.bytes = 0;
+    CUDA_TRY(cudaMalloc(&w.base, need));
+    w.bytes = need;
+    CUDA_TRY(cudaMemset(w.base, 0, need));
+  }
+  if (!(w.shape == s)) {
+    layout(s, &w, static_cast<char*>(w.base));
+    w.shape = s;
+    w.stage = 0;
+  }
+  *out = &w;
+  return SOL_ATTN_OK;
+}
+
+int check_shape(int B, int H, int L, int d, int block) {
+  if (B <= 0 || H <= 0 || L <= 0) return fail(SOL_ATTN_ERR_ARG, "B, H, L must be positive (got %d, %d, %d)", B, H, L);
+  if (block != kBlock) return fail(SOL_ATTN_ERR_UNSUPPORTED, "block must be 64 (got %d)", block);
+  if (d != 64 && d != 128) return fail(SOL_ATTN_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+  if (L > kMaxL) return fail(SOL_ATTN_ERR_UNSUPPORTED, "L = %d exceeds the supported maximum %d", L, kMaxL);
+  if (static_cast<long long>(B) * H > (1LL << 24)) return fail(SOL_ATTN_ERR_UNSUPPORTED, "B*H too large");
+  return SOL_ATTN_OK;
+}
+
+int check_ptr(const void* p, const char* name) {
+  if (!p) return fail(SOL_ATTN_ERR_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return fail(SOL_ATTN_ERR_ALIGN, "%s is not 16-byte aligned", name);
+  return SOL_ATTN_OK;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encoder(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) return fail(SOL_ATTN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *fn = cached;
+  return SOL_ATTN_OK;
+}
+
+// 3-D bf16 map over [BH][rows][d] with a {64, box_rows, 1} box and 128-byte swizzle.
+// Rows past `rows` read as zero.
+int make_map(CUtensorMap* m, const void* ptr, int d, long long rows, long long BH, int box_rows) {
+  EncodeTiledFn enc;
+  int rc = get_encoder(&enc);
+  if (rc) return rc;
+  cuuint64_t gdim[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(BH)};
+  cuuint64_t gstride[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), gdim, gstride, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SOL_ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SOL_ATTN_OK;
+}
+
+// ------------------------------------------------------------------ stages
+int run_pool(Workspace& w, const void* q, const void* k, const void* v, const sol_attn_debug* dbg,
+             cudaStream_t st) {
+  const Shape& s = w.shape;
+  const int N = (s.L + kBlock - 1) / kBlock;
+  dim3 grid(N, s.B * s.H);
+  float* vdbg = dbg ? dbg->vhat : nullptr;
+  auto qq = static_cast<const uint16_t*>(q);
+  auto kk = static_cast<const uint16_t*>(k);
+  auto vv = static_cast<const uint16_t*>(v);
+  if (s.d == 128)
+    pool_kernel<128><<<grid, 256, 0, st>>>(qq, kk, vv, s.L, N, w.qbar, w.kbar, w.kbar_bf, w.kbar_lo, w.vhat_bf,
+                                           vdbg);
+  else
+    pool_kernel<64><<<grid, 256, 0, st>>>(qq, kk, vv, s.L, N, w.qbar, w.kbar, w.kbar_bf, w.kbar_lo, w.vhat_bf,
+                                          vdbg);
+  CUDA_TRY(cudaGetLastError());
+  const size_t nbytes = static_cast<size_t>(s.B) * s.H * N * s.d * 4;
+  if (dbg && dbg->qbar) CUDA_TRY(cudaMemcpyAsync(dbg->qbar, w.qbar, nbytes, cudaMemcpyDeviceToDevice, st));
+  if (dbg && dbg->kbar) CUDA_TRY(cudaMemcpyAsync(dbg->kbar, w.kbar, nbytes, cudaMemcpyDeviceToDevice, st));
+  w.stage = 1;
+  return SOL_ATTN_OK;
+}
+
+template <int D>
+int launch_threshold(Workspace& w, int N, float beta, int mode, const sol_attn_debug* dbg, cudaStream_t st) {
+  const int BH = w.shape.B * w.shape.H;
+  moments_kernel<D><<<BH, 256, 0, st>>>(w.kbar, N, w.mom_mean, w.mom_cov);
+  CUDA_TRY(cudaGetLastError());
+  const size_t smem = (static_cast<size_t>(D) * D + D + 8 * 4 * D) * sizeof(double);
+  static bool attr_set = false;
+  if (!attr_set) {
+    CUDA_TRY(cudaFuncSetAttribute(threshold_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(smem)));
+    attr_set = true;
+  }
+  dim3 grid((N + 31) / 32, BH);
+  threshold_kernel<D><<<grid, 256, smem, st>>>(w.qbar, w.mom_mean, w.mom_cov, N, beta, mode, w.tau,
+                                                dbg ? dbg->mu : nullptr, dbg ? dbg->sigma : nullptr);
+  CUDA_TRY(cudaGetLastError());
+  return SOL_ATTN_OK;
+}
+
+int run_threshold(Workspace& w, float beta, unsigned flags, const sol_attn_debug* dbg, cudaStream_t st) {
+  const Shape& s = w.shape;
+  const int N = (s.L + kBlock - 1) / kBlock;
+  int mode = kThresholdBeta;
+  if ((flags & SOL_ATTN_FLAG_SELECT_ALL) || (std::isinf(beta) && beta < 0)) mode = kThresholdSelectAll;
+  else if (std::isinf(beta)) mode = kThresholdSelectNone;
+  int rc = (s.d == 128) ? launch_threshold<128>(w, N, beta, mode, dbg, st)
+                        : launch_threshold<64>(w, N, beta, mode, dbg, st);
+  if (rc) return rc;
+  if (dbg && dbg->tau)
+    CUDA_TRY(cudaMemcpyAsync(dbg->tau, w.tau, static_cast<size_t>(s.B) * s.H * N * 4, cudaMemcpyDeviceToDevice, st));
+  w.stage = 2;
+  return SOL_ATTN_OK;
+}
+
+template <int D>
+int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void* out, int chunk, unsigned flags,
+                 const sol_attn_debug* dbg, cudaStream_t st) {
+  const Shape& s = w.shape;
+  const int N = (s.L + kBlock - 1) / kBlock;
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  if ((N + 31) / 32 > kMaxMaskWords)
+    return fail(SOL_ATTN_ERR_UNSUPPORTED, "N = %d pooled blocks exceeds the fused kernel's %d", N, kMaxMaskWords * 32);
+  const int W = std::min(64, (std::min(chunk, N) + 31) / 32 * 32);
+  CUtensorMap tq, tk, tv, tkb, tkl, tvb;
+  int rc;
+  if ((rc = make_map(&tq, q, D, s.L, BH, 128))) return rc;
+  if ((rc = make_map(&tk, k, D, s.L, BH, 64))) return rc;
+  if ((rc = make_map(&tv, v, D, s.L, BH, 64))) return rc;
+  if ((rc = make_map(&tkb, w.kbar_bf, D, N, BH, W))) return rc;
+  if ((rc = make_map(&tkl, w.kbar_lo, D, N, BH, W))) return rc;
+  if ((rc = make_map(&tvb, w.vhat_bf, D, N, BH, W))) return rc;
+
+  FusedParams p{};
+  p.BH = static_cast<int>(BH);
+  p.L = s.L;
+  p.N = N;
+  p.W = W;
+  p.chunk = chunk;
+  p.num_pairs = (N + 1) / 2;
+  p.num_items = static_cast<int>(BH * p.num_pairs);
+  p.flags = flags;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  p.qbar = w.qbar;
+  p.kbar = w.kbar;
+  p.tau = w.tau;
+  p.counts = w.counts;
+  p.mask_out = dbg ? dbg->mask : nullptr;
+  p.out = static_cast<uint16_t*>(out);
+  p.work_counter = w.counter;
+  p.status = w.status;
+  p.timeout_ns = kTimeoutNs;
+
+  int dev = 0, nsm = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+  static bool attr_set = false;
+  if (!attr_set) {
+    CUDA_TRY(cudaFuncSetAttribute(sol_attn_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kFusedSmemBytes)));
+    attr_set = true;
+  }
+  CUDA_TRY(cudaMemsetAsync(w.counter, 0, sizeof(unsigned), st));
+  const int grid = std::min(p.num_items, nsm);
+  sol_attn_fused_kernel<D><<<grid, 128, kFusedSmemBytes, st>>>(tq, tk, tv, tkb, tkl, tvb, p);
+  CUDA_TRY(cudaGetLastError());
+  return SOL_ATTN_OK;
+}
+
+int run_fused(Workspace& w, const void* q, const void* k, const void* v, void* out, int chunk, unsigned flags,
+              const sol_attn_debug* dbg, cudaStream_t st) {
+  int rc = (w.shape.d == 128) ? launch_fused<128>(w, q, k, v, out, chunk, flags, dbg, st)
+                              : launch_fused<64>(w, q, k, v, out, chunk, flags, dbg, st);
+  if (rc) return rc;
+  w.stage = 3;
+  w.last_fused = w.shape;
+  return SOL_ATTN_OK;
+}
+
+int read_status(Workspace& w, cudaStream_t st) {
+  CUDA_TRY(cudaStreamSynchronize(st));
+  unsigned h = 0;
+  CUDA_TRY(cudaMemcpy(&h, w.status, sizeof(h), cudaMemcpyDeviceToHost));
+  if (h) {
+    CUDA_TRY(cudaMemset(w.status, 0, sizeof(unsigned)));
+    if (h & kStatusTimeout) return fail(SOL_ATTN_ERR_TIMEOUT, "a bounded device wait gave up (status 0x%x)", h);
+    return fail(SOL_ATTN_ERR_DEVICE, "device-side check failed (status 0x%x)", h);
+  }
+  return SOL_ATTN_OK;
+}
+
+int check_io(const void* q, const void* k, const void* v, const void* out, int B, int H, int L, int d) {
+  int rc;
+  if ((rc = check_ptr(q, "q")) || (rc = check_ptr(k, "k")) || (rc = check_ptr(v, "v"))) return rc;
+  if (out) {
+    if ((rc = check_ptr(out, "out"))) return rc;
+    const size_t n = static_cast<size_t>(B) * H * L * d * 2;
+    const char* o = static_cast<const char*>(out);
+    for (const void* x : {q, k, v}) {
+      const char* xc = static_cast<const char*>(x);
+      if (o < xc + n && xc < o + n) return fail(SOL_ATTN_ERR_ARG, "out overlaps an input tensor");
+    }
+  }
+  return SOL_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, int B, int H, int L, int d, int block,
+                        int chunk, float beta, unsigned flags, const sol_attn_debug* dbg, void* stream) {
+  int rc;
+  if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if (chunk < 1) return fail(SOL_ATTN_ERR_ARG, "chunk must be >= 1 (got %d)", chunk);
+  if (std::isnan(beta)) return fail(SOL_ATTN_ERR_ARG, "beta is NaN");
+  if (!out) return fail(SOL_ATTN_ERR_ARG, "out is NULL");
+  if ((rc = check_io(q, k, v, out, B, H, L, d))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace* w;
+  if ((rc = ensure_ws(Shape{B, H, L, d}, &w))) return rc;
+  auto st = static_cast<cudaStream_t>(stream);
+  if ((rc = run_pool(*w, q, k, v, dbg, st))) return rc;
+  if ((rc = run_threshold(*w, beta, flags, dbg, st))) return rc;
+  if ((rc = run_fused(*w, q, k, v, out, chunk, flags, dbg, st))) return rc;
+  if (flags & SOL_ATTN_FLAG_SYNC_CHECK) return read_status(*w, st);
+  return SOL_ATTN_OK;
+}
+
+int sol_attn_forward(const void* q, const void* k, const void* v, void* out, int B, int H, int L, int d, int block,
+                     int chunk, float beta, void* stream) {
+  return sol_attn_forward_ex(q, k, v, out, B, H, L, d, block, chunk, beta, 0u, nullptr, stream);
+}
+
+int sol_attn_stage_pool(const void* q, const void* k, const void* v, int B, int H, int L, int d, int block,
+                        const sol_attn_debug* dbg, void* stream) {
+  int rc;
+  if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if ((rc = check_io(q, k, v, nullptr, B, H, L, d))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace* w;
+  if ((rc = ensure_ws(Shape{B, H, L, d}, &w))) return rc;
+  return run_pool(*w, q, k, v, dbg, static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_stage_threshold(int B, int H, int L, int d, int block, float beta, unsigned flags,
+                             const sol_attn_debug* dbg, void* stream) {
+  int rc;
+  if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if (std::isnan(beta)) return fail(SOL_ATTN_ERR_ARG, "beta is NaN");
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  Workspace& w = g_ws[dev];
+  if (!(w.shape == Shape{B, H, L, d}) || w.stage < 1)
+    return fail(SOL_ATTN_ERR_STATE, "stage_threshold needs a stage_pool of the same shape first");
+  return run_threshold(w, beta, flags, dbg, static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_stage_fused(const void* q, const void* k, const void* v, void* out, int B, int H, int L, int d, int block,
+                         int chunk, unsigned flags, const sol_attn_debug* dbg, void* stream) {
+  int rc;
+  if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if (chunk < 1) return fail(SOL_ATTN_ERR_ARG, "chunk must be >= 1 (got %d)", chunk);
+  if (!out) return fail(SOL_ATTN_ERR_ARG, "out is NULL");
+  if ((rc = check_io(q, k, v, out, B, H, L, d))) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  Workspace& w = g_ws[dev];
+  if (!(w.shape == Shape{B, H, L, d}) || w.stage < 2)
+    return fail(SOL_ATTN_ERR_STATE, "stage_fused needs stage_pool and stage_threshold of the same shape first");
+  auto st = static_cast<cudaStream_t>(stream);
+  if ((rc = run_fused(w, q, k, v, out, chunk, flags, dbg, st))) return rc;
+  if (flags & SOL_ATTN_FLAG_SYNC_CHECK) return read_status(w, st);
+  return SOL_ATTN_OK;
+}
+
+int sol_attn_stats(int32_t* counts, int B, int H, int L, int block, void* stream) {
+  if (!counts) return fail(SOL_ATTN_ERR_ARG, "counts is NULL");
+  if (B <= 0 || H <= 0 || L <= 0) return fail(SOL_ATTN_ERR_ARG, "B, H, L must be positive");
+  if (block != kBlock) return fail(SOL_ATTN_ERR_UNSUPPORTED, "block must be 64 (got %d)", block);
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  Workspace& w = g_ws[dev];
+  const Shape& f = w.last_fused;
+  if (w.stage < 3 || f.B != B || f.H != H || f.L != L || !(w.shape == f))
+    return fail(SOL_ATTN_ERR_STATE, "no forward of shape (B=%d, H=%d, L=%d) to report on", B, H, L);
+  const size_t N = (static_cast<size_t>(L) + kBlock - 1) / kBlock;
+  CUDA_TRY(cudaMemcpyAsync(counts, w.counts, static_cast<size_t>(B) * H * N * sizeof(int32_t),
+                           cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return SOL_ATTN_OK;
+}
+
+int sol_attn_forward_host(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int B, int H, int L,
+                          int d, int block, int chunk, float beta, unsigned flags) {
+  int rc;
+  if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if (!q || !k || !v || !out) return fail(SOL_ATTN_ERR_ARG, "a host pointer is NULL");
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  const size_t n = static_cast<size_t>(B) * H * L * d * 2;
+  const size_t per = align_up(n, 256);
+  char* dq;
+  cudaStream_t st;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace& w = g_ws[dev];
+    if (!w.host_stream) CUDA_TRY(cudaStreamCreateWithFlags(&w.host_stream, cudaStreamNonBlocking));
+    if (w.host_stage_bytes < 4 * per) {
+      if (w.host_stage) CUDA_TRY(cudaFree(w.host_stage));
+      w.host_stage = nullptr;
+      w.host_stage_bytes = 0;
+      CUDA_TRY(cudaMalloc(&w.host_stage, 4 * per));
+      w.host_stage_bytes = 4 * per;
+    }
+    dq = static_cast<char*>(w.host_stage);
+    st = w.host_stream;
+  }
+  CUDA_TRY(cudaMemcpyAsync(dq, q, n, cudaMemcpyHostToDevice, st));
+  CUDA_TRY(cudaMemcpyAsync(dq + per, k, n, cudaMemcpyHostToDevice, st));
+  CUDA_TRY(cudaMemcpyAsync(dq + 2 * per, v, n, cudaMemcpyHostToDevice, st));
+  rc = sol_attn_forward_ex(dq, dq + per, dq + 2 * per, dq + 3 * per, B, H, L, d, block, chunk, beta,
+                           flags & ~SOL_ATTN_FLAG_SYNC_CHECK, nullptr, st);
+  if (rc) return rc;
+  CUDA_TRY(cudaMemcpyAsync(out, dq + 3 * per, n, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  if (flags & SOL_ATTN_FLAG_SYNC_CHECK) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return read_status(g_ws[dev], st);
+  }
+  return SOL_ATTN_OK;
+}
+
+size_t sol_attn_workspace_bytes(int B, int H, int L, int d, int block) {
+  if (check_shape(B, H, L, d, block)) return 0;
+  return layout(Shape{B, H, L, d}, nullptr, nullptr);
+}
+
+int sol_attn_release(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  Workspace& w = g_ws[dev];
+  if (w.base) CUDA_TRY(cudaFree(w.base));
+  if (w.ctl_block) CUDA_TRY(cudaFree(w.ctl_block));
+  if (w.host_stage) CUDA_TRY(cudaFree(w.host_stage));
+  if (w.host_stream) CUDA_TRY(cudaStreamDestroy(w.host_stream));
+  w = Workspace{};
+  return SOL_ATTN_OK;
+}
+
+const char* sol_attn_error_string(int code) {
+  static thread_local std::string msg;
+  const char* base = "unknown status";
+  switch (code) {
+    case SOL_ATTN_OK: base = "ok"; break;
+    case SOL_ATTN_ERR_ARG: base = "invalid argument"; break;
+    case SOL_ATTN_ERR_UNSUPPORTED: base = "unsupported configuration"; break;
+    case SOL_ATTN_ERR_ALIGN: base = "misaligned pointer"; break;
+    case SOL_ATTN_ERR_CUDA: base = "CUDA error"; break;
+    case SOL_ATTN_ERR_TIMEOUT: base = "device wait timed out"; break;
+    case SOL_ATTN_ERR_STATE: base = "invalid call order / state"; break;
+    case SOL_ATTN_ERR_DEVICE: base = "device-side check failed"; break;
+  }
+  msg = base;
+  if (code != SOL_ATTN_OK && !g_last_error.empty()) msg += ": " + g_last_error;
+  return msg.c_str();
+}
+
+int sol_attn_kernels_per_forward(void) { return 4; }
+
+}  // extern "C"

@@ -1,0 +1,137 @@
+/*
+ * sol_attn.h — C ABI of the Sol-Attn single-pass sparse attention forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "Sol-Attn: Accelerating Video Generation Inference via On-the-Fly
+ * Attention Sparsification".  For every query block i of 64 tokens the forward
+ *   1. mean-pools 64-token blocks into Q̄_i, K̄_j and sums values into V̂_j
+ *      (method: threshold routing, Eq. 3; proxy-score reuse, V̂ before Eq. 9);
+ *   2. derives τ_i = μ_i + β σ_i from the first and second moments of the
+ *      pooled keys, never forming the N x N proxy map (Eq. 4-5);
+ *   3. in one online-softmax pass scans the pooled keys in chunks of C, selects
+ *      block j when ŝ_ij = Q̄_i·K̄_j/sqrt(d) >= τ_i (Eq. 6-7), runs exact
+ *      attention over the selected K/V blocks, and adds the zeroth-order
+ *      approximation exp(q_r·K̄_j/sqrt(d)) for every unselected block, weighted
+ *      by its token count n_j in the denominator and applied to V̂_j in the
+ *      numerator (Eq. 8-10, batched as the token-to-block tile of Eq. 11).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors q, k, v, out are contiguous row-major [B, H, L, d] bf16 (raw
+ *     16-bit patterns), device memory unless stated otherwise, each base
+ *     address 16-byte aligned.  out must not overlap q, k or v.
+ *   - block must be 64 (fixed 64x64 physical blocks, experiments: setup);
+ *     d must be 64 or 128; N = ceil(L / 64); the last block may be ragged and
+ *     is pooled over its valid tokens.  1 <= L <= 1,048,576, chunk >= 1.
+ *   - beta: any finite value; -INFINITY selects every block (dense mode),
+ *     +INFINITY selects none (every block approximated); NaN is rejected.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued without a host synchronisation unless a flag asks for
+ *     one; errors detected while enqueuing are returned immediately.
+ *   - The library owns a per-device workspace (pooled tensors, thresholds,
+ *     per-row counts, a work counter and a status word) that grows on demand
+ *     with cudaMalloc; the first call for a larger shape therefore must not be
+ *     inside a stream capture.  Calls on one device share the workspace: do
+ *     not run two forwards concurrently on different streams of one device.
+ *   - Return value: SOL_ATTN_OK (0) or a negative sol_attn_status code.
+ *     sol_attn_error_string() describes the last error in words.
+ */
+#ifndef SOL_ATTN_H_
+#define SOL_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sol_attn_status {
+  SOL_ATTN_OK = 0,
+  SOL_ATTN_ERR_ARG = -1,          /* null pointer, non-positive size, NaN beta, chunk < 1 */
+  SOL_ATTN_ERR_UNSUPPORTED = -2,  /* d not in {64,128}, block != 64, L too large, not sm_100 */
+  SOL_ATTN_ERR_ALIGN = -3,        /* a tensor base address is not 16-byte aligned */
+  SOL_ATTN_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
+  SOL_ATTN_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up (status word) */
+  SOL_ATTN_ERR_STATE = -6,        /* stats/stage call without a matching earlier forward */
+  SOL_ATTN_ERR_DEVICE = -7        /* a device-side consistency check failed (status word) */
+} sol_attn_status;
+
+/* Flags for sol_attn_forward_ex. */
+#define SOL_ATTN_FLAG_SELECT_ALL 0x1u  /* ignore beta; select every block (dense baseline) */
+#define SOL_ATTN_FLAG_EXACT_ONLY 0x2u  /* keep-or-drop: skip the approximation of unselected
+                                          blocks (ablation: exact-only vs exact-or-approx) */
+#define SOL_ATTN_FLAG_SYNC_CHECK 0x4u  /* synchronise the stream after the forward and read
+                                          the device status word (timeouts, device checks) */
+
+/* Optional device buffers filled by sol_attn_forward_ex (any member may be NULL).
+ * Shapes use N = ceil(L/64); all are row-major and owned by the caller. */
+typedef struct sol_attn_debug {
+  float* qbar;     /* [B,H,N,d] pooled queries Q̄ (mean over valid tokens), fp32 */
+  float* kbar;     /* [B,H,N,d] pooled keys K̄, fp32 */
+  float* vhat;     /* [B,H,N,d] summed values V̂ (sum over valid tokens), fp32 */
+  float* mu;       /* [B,H,N] proxy-row mean μ_i from the key moments */
+  float* sigma;    /* [B,H,N] proxy-row standard deviation σ_i from the key moments */
+  float* tau;      /* [B,H,N] threshold τ_i (±inf in select-all / select-none) */
+  uint32_t* mask;  /* [B,H,N,ceil(N/32)] selection bits: block j of row i is bit (j%32)
+                      of word j/32; written by the fused kernel's routing step */
+} sol_attn_debug;
+
+/* Sol-Attn forward (method: Eq. 3-11).  q, k, v: input [B,H,L,d] bf16 device
+ * tensors; out: output [B,H,L,d] bf16 device tensor, every valid row written.
+ * chunk: C, the number of pooled keys routed per outer-loop step (Eq. 6); it
+ * changes the schedule, not the result.  Enqueues three kernels (pool,
+ * moments, fused attention) on stream. */
+int sol_attn_forward(const void* q, const void* k, const void* v, void* out,
+                     int B, int H, int L, int d, int block, int chunk, float beta,
+                     void* stream);
+
+/* As sol_attn_forward, with SOL_ATTN_FLAG_* flags and optional debug exports
+ * (dbg may be NULL). */
+int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out,
+                        int B, int H, int L, int d, int block, int chunk, float beta,
+                        unsigned flags, const sol_attn_debug* dbg, void* stream);
+
+/* Per-row selected-block counts |S_i| (density analysis, ablation: Fig. 7):
+ * copies the [B,H,N] int32 counts written by the last forward on this device
+ * into counts (device memory), enqueued on stream.  Returns SOL_ATTN_ERR_STATE
+ * if the last forward had a different (B,H,L,block). */
+int sol_attn_stats(int32_t* counts, int B, int H, int L, int block, void* stream);
+
+/* End-to-end call on HOST buffers (pinned or pageable): copies q, k, v to the
+ * device, runs sol_attn_forward_ex on an internal stream, copies out back and
+ * synchronises.  Device staging buffers are owned and cached by the library. */
+int sol_attn_forward_host(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          uint16_t* out, int B, int H, int L, int d, int block,
+                          int chunk, float beta, unsigned flags);
+
+/* The three stages of sol_attn_forward_ex as separate calls on one stream, for
+ * per-kernel timing and staged checks.  They must be called in this order with
+ * the same shape; a later stage returns SOL_ATTN_ERR_STATE otherwise.
+ *   stage_pool:      block pooling of q, k, v into the workspace (method: Eq. 3, V̂).
+ *   stage_threshold: key moments and τ_i = μ_i + β σ_i (Eq. 4-5).
+ *   stage_fused:     routing, exact inner loop and approximation (Eq. 6-11). */
+int sol_attn_stage_pool(const void* q, const void* k, const void* v, int B, int H, int L,
+                        int d, int block, const sol_attn_debug* dbg, void* stream);
+int sol_attn_stage_threshold(int B, int H, int L, int d, int block, float beta,
+                             unsigned flags, const sol_attn_debug* dbg, void* stream);
+int sol_attn_stage_fused(const void* q, const void* k, const void* v, void* out, int B,
+                         int H, int L, int d, int block, int chunk, unsigned flags,
+                         const sol_attn_debug* dbg, void* stream);
+
+/* Bytes of device workspace the library holds for this shape. */
+size_t sol_attn_workspace_bytes(int B, int H, int L, int d, int block);
+
+/* Frees the calling thread's current-device workspace (no work may be in flight). */
+int sol_attn_release(void);
+
+/* Text for a status code, including detail of the most recent failure. */
+const char* sol_attn_error_string(int code);
+
+/* Number of kernels one sol_attn_forward enqueues (for launch accounting). */
+int sol_attn_kernels_per_forward(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_ATTN_H_ */

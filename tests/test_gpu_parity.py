@@ -1,0 +1,165 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+identical seeded bf16 inputs, for the five workload shapes and the edge cases.
+
+"Sol-Attn: Accelerating Video Generation Inference via On-the-Fly Attention
+Sparsification": masks follow Eq. 4 / Eq. 6-7, outputs Eq. 9-10."""
+import math
+
+import numpy as np
+import pytest
+
+import block_sparse_attention_moments_b200 as sa
+from parity_util import Report, compare_head, debug_numpy, run_gpu
+from synth import WORKLOADS, custom_fourier, fourier_inputs, gauss_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    sa.lib()
+
+
+def _full_check(qb, kb, vb, beta, chunk, flags=0, heads=None, rows=None):
+    out, dbg, counts = run_gpu(qb, kb, vb, beta, chunk, flags=flags)
+    sel = dbg.selection().cpu().numpy()
+    dn = debug_numpy(dbg)
+    rep = Report()
+    B, H = qb.shape[:2]
+    for bh in (range(B * H) if heads is None else heads):
+        b, h = divmod(bh, H)
+        compare_head(rep, qb, kb, vb, b, h, beta, out, sel, counts, rows=rows,
+                     exact_only=bool(flags & sa.FLAG_EXACT_ONLY), dbg=dn)
+    print(rep)
+    rep.check()
+    return out, sel, rep
+
+
+@pytest.mark.parametrize("beta", [1.0, 0.5, 1.5, -math.inf, math.inf])
+def test_tiny_shape(beta):
+    wl = WORKLOADS["tiny"]
+    qb, kb, vb = fourier_inputs(wl)
+    _full_check(qb, kb, vb, beta, wl.chunk)
+
+
+@pytest.mark.parametrize("beta", [0.5, 1.0, 1.5, -math.inf])
+def test_small_shape(beta):
+    wl = WORKLOADS["small"]
+    qb, kb, vb = fourier_inputs(wl)
+    _full_check(qb, kb, vb, beta, wl.chunk)
+
+
+def test_chunk_size_does_not_change_the_result():
+    # experiments: setup — C affects efficiency, not the output
+    wl = WORKLOADS["small"]
+    qb, kb, vb = fourier_inputs(wl)
+    ref_out, ref_sel, _ = _full_check(qb, kb, vb, 1.0, wl.chunk)
+    for C in (1, 3, 7, 32, 64, 100, 500):
+        out, sel, _ = _full_check(qb, kb, vb, 1.0, C)
+        assert (sel == ref_sel).all()
+        assert np.abs(out - ref_out).max() <= 2e-2
+
+
+def test_select_all_flag_equals_dense_beta():
+    wl = WORKLOADS["small"]
+    qb, kb, vb = fourier_inputs(wl)
+    a, _, _ = run_gpu(qb, kb, vb, 1.0, wl.chunk, flags=sa.FLAG_SELECT_ALL, debug=False)
+    b, _, _ = run_gpu(qb, kb, vb, -math.inf, wl.chunk, debug=False)
+    assert np.array_equal(a, b)
+    _full_check(qb, kb, vb, -math.inf, wl.chunk, flags=sa.FLAG_SELECT_ALL)
+
+
+@pytest.mark.parametrize("beta", [0.5, 1.0, math.inf])
+def test_exact_only_flag(beta):
+    wl = WORKLOADS["small"]
+    qb, kb, vb = fourier_inputs(wl)
+    _full_check(qb, kb, vb, beta, wl.chunk, flags=sa.FLAG_EXACT_ONLY)
+
+
+def test_image_shape():
+    wl = WORKLOADS["image"]
+    qb, kb, vb = fourier_inputs(wl)
+    B, H = wl.B, wl.H
+    # three heads in full, and sampled query blocks of every other head
+    full = [0, H + 7, B * H - 1]
+    _full_check(qb, kb, vb, 1.0, wl.chunk, heads=full)
+    rng = np.random.default_rng(5)
+    rows = sorted(set(rng.integers(0, wl.N, size=6).tolist()) | {0, wl.N - 1})
+    _full_check(qb, kb, vb, 1.0, wl.chunk, heads=[bh for bh in range(B * H) if bh not in full][::5], rows=rows)
+
+
+@pytest.mark.parametrize("name,beta", [("wan", 1.0), ("wan", 0.75), ("wan", 1.5), ("hunyuan", 1.0),
+                                       ("hunyuan", -math.inf)])
+def test_video_shapes_sampled(name, beta):
+    # full-size launch (the bench's configuration); oracle on sampled query
+    # blocks of sampled heads, always including the ragged last block
+    wl = WORKLOADS[name]
+    qb, kb, vb = fourier_inputs(wl)
+    rng = np.random.default_rng(11)
+    heads = sorted(set(rng.integers(0, wl.B * wl.H, size=3).tolist()) | {wl.B * wl.H - 1})
+    rows = sorted(set(rng.integers(0, wl.N, size=4).tolist()) | {0, wl.N - 2, wl.N - 1})
+    _full_check(qb, kb, vb, beta, wl.chunk, heads=heads, rows=rows)
+
+
+@pytest.mark.parametrize("L,d,chunk", [(1, 128, 4), (64, 128, 1), (65, 64, 2), (127, 128, 4), (129, 64, 3),
+                                       (1000, 128, 5), (4033, 64, 16), (4096, 128, 200)])
+@pytest.mark.parametrize("beta", [0.75, -math.inf, math.inf])
+def test_edge_shapes(L, d, chunk, beta):
+    qb, kb, vb = custom_fourier(2, 2, (1, 1, L), d, 2.0, seed=L * 7 + d)
+    _full_check(qb, kb, vb, beta, chunk)
+
+
+def test_gaussian_inputs_density():
+    qb, kb, vb = gauss_inputs(1, 2, 64 * 512, 128, seed=12)
+    for beta, rho in ((0.5, 0.3085), (1.0, 0.1587), (1.5, 0.0668)):
+        out, sel, rep = _full_check(qb, kb, vb, beta, 64, rows=list(range(0, 512, 37)) + [511])
+        _, _, counts = run_gpu(qb, kb, vb, beta, 64, debug=False)
+        assert abs(counts.mean() / 512 - rho) < 0.01
+
+
+def test_host_buffer_entry_point_matches_device_call():
+    wl = WORKLOADS["small"]
+    qb, kb, vb = fourier_inputs(wl)
+    dev, _, _ = run_gpu(qb, kb, vb, 1.0, wl.chunk, debug=False)
+    host = sa.forward_host(qb, kb, vb, 1.0, wl.chunk, flags=sa.FLAG_SYNC_CHECK)
+    import torch
+    got = torch.from_numpy(host.view(np.int16)).view(torch.bfloat16).float().numpy()
+    assert np.array_equal(got, dev)
+
+
+def test_staged_calls_match_forward():
+    import torch
+    from parity_util import to_device
+    wl = WORKLOADS["small"]
+    qb, kb, vb = fourier_inputs(wl)
+    ref, _, _ = run_gpu(qb, kb, vb, 1.0, wl.chunk, debug=False)
+    q, k, v = to_device(qb), to_device(kb), to_device(vb)
+    out = torch.empty_like(q)
+    sa.stage_pool(q, k, v)
+    sa.stage_threshold(wl.B, wl.H, wl.L, wl.d, 1.0)
+    sa.stage_fused(q, k, v, out, wl.chunk, flags=sa.FLAG_SYNC_CHECK)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.float().cpu().numpy(), ref)
+
+
+def test_runtime_errors_on_device():
+    import torch
+    from parity_util import to_device
+    wl = WORKLOADS["tiny"]
+    qb, kb, vb = fourier_inputs(wl)
+    q, k, v = to_device(qb), to_device(kb), to_device(vb)
+    flat = torch.empty(q.numel() + 8, dtype=torch.bfloat16, device="cuda")
+    mis = flat[1:1 + q.numel()].view(q.shape)       # 2-byte offset: misaligned
+    with pytest.raises(sa.SolAttnError) as e:
+        sa.forward(mis, k, v, 1.0, 4)
+    assert e.value.code == -3
+    sa.forward(q, k, v, 1.0, 4)
+    with pytest.raises(sa.SolAttnError) as e:
+        sa.stats(1, 1, 2048)                          # no forward of that shape
+    assert e.value.code == -6
+    with pytest.raises(sa.SolAttnError) as e:
+        sa.stage_fused(q, k, v, torch.empty_like(q), 4) if False else sa.stage_threshold(1, 3, 1024, 64, 1.0)
+    assert e.value.code == -6
