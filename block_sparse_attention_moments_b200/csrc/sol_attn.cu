@@ -364,6 +364,35 @@ int check_io(const void* q, const void* k, const void* v, const void* out, int B
   return SOL_ATTN_OK;
 }
 
+// ------------------------------------------------------------------ allocation-free forward
+// Some callers cannot call cudaMalloc: code running inside a custom or
+// pre-reserved memory pool that forbids outside allocations, latency-critical
+// serving loops where an allocation could synchronise the device, and hosts
+// that hand this library only the tensors it reads and writes.  For them the
+// scratch of sol_attn_forward_noalloc lives in this fixed device array,
+// reserved once per GPU when the library is loaded and held until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(96) << 20;   // 96 MiB
+constexpr size_t kNoAllocCtlBytes = 256;                    // work counter + status word
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device with that
+// device current (the host-side symbol is only a stand-in, not an address).
+char* g_noalloc_base[kMaxDevices] = {nullptr};
+
+int noalloc_base(int dev, char** out) {
+  if (!g_noalloc_base[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return fail(SOL_ATTN_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    // the status word must start at zero; the work counter is cleared before every launch
+    CUDA_TRY(cudaMemset(ptr, 0, kNoAllocCtlBytes));
+    g_noalloc_base[dev] = static_cast<char*>(ptr);
+  }
+  *out = g_noalloc_base[dev];
+  return SOL_ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -530,5 +559,39 @@ const char* sol_attn_error_string(int code) {
 }
 
 int sol_attn_kernels_per_forward(void) { return 4; }
+
+int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int H, int L, int d,
+                             int block, int chunk, float beta, void* stream) {
+  int rc;
+  if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if (chunk < 1) return fail(SOL_ATTN_ERR_ARG, "chunk must be >= 1 (got %d)", chunk);
+  if (std::isnan(beta)) return fail(SOL_ATTN_ERR_ARG, "beta is NaN");
+  if (!out) return fail(SOL_ATTN_ERR_ARG, "out is NULL");
+  if ((rc = check_io(q, k, v, out, B, H, L, d))) return rc;
+  const Shape s{B, H, L, d};
+  const size_t need = layout(s, nullptr, nullptr);
+  if (need > kNoAllocScratchBytes - kNoAllocCtlBytes)
+    return fail(SOL_ATTN_ERR_UNSUPPORTED,
+                "shape (B=%d, H=%d, L=%d, d=%d) needs %zu bytes of scratch; the allocation-free entry point "
+                "holds %zu",
+                B, H, L, d, need, kNoAllocScratchBytes - kNoAllocCtlBytes);
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  if ((rc = check_arch(dev))) return rc;
+  char* base;
+  if ((rc = noalloc_base(dev, &base))) return rc;
+  Workspace w;   // a view over the fixed array; nothing is allocated
+  w.counter = reinterpret_cast<unsigned*>(base);
+  w.status = reinterpret_cast<unsigned*>(base) + 32;
+  w.base = base + kNoAllocCtlBytes;
+  w.bytes = kNoAllocScratchBytes - kNoAllocCtlBytes;
+  layout(s, &w, static_cast<char*>(w.base));
+  w.shape = s;
+  auto st = static_cast<cudaStream_t>(stream);
+  if ((rc = run_pool(w, q, k, v, nullptr, st))) return rc;
+  if ((rc = run_threshold(w, beta, 0u, nullptr, st))) return rc;
+  return run_fused(w, q, k, v, out, chunk, 0u, nullptr, st);
+}
 
 }  // extern "C"

@@ -130,6 +130,23 @@ const char* sol_attn_error_string(int code);
 /* Number of kernels one sol_attn_forward enqueues (for launch accounting). */
 int sol_attn_kernels_per_forward(void);
 
+/* Allocation-free variant of sol_attn_forward (the paper has no counterpart;
+ * it exists for callers that may not allocate device memory, e.g. code inside
+ * a fixed memory pool or a serving loop where cudaMalloc could synchronise).
+ * Same arguments, layout and result as sol_attn_forward.  Its scratch lives in
+ * one fixed 96 MiB device array inside the library, reserved on every GPU that
+ * loads it and held until the process exits; shapes whose scratch does not fit
+ * (about B*H*ceil(L/64)*d*14 + B*H*d*d*8 bytes) return SOL_ATTN_ERR_UNSUPPORTED.
+ * Nothing is allocated or freed.  The first call on a device looks up that
+ * array's device address and clears its status word, so make that first call
+ * outside any stream capture.  All calls on a device share the array and it
+ * keeps the last call's contents: calls that overlap on the GPU (different
+ * streams, or host threads racing) race on it and must be serialised by the
+ * caller.  sol_attn_stats does not report on these calls. */
+int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out,
+                             int B, int H, int L, int d, int block, int chunk, float beta,
+                             void* stream);
+
 #ifdef __cplusplus
 }
 #endif
