@@ -221,6 +221,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=768, help="query blocks in the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the select-all (dense) comparison run")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -287,7 +288,10 @@ def main():
     # sparse run (the headline) and the same kernel in select-all (dense) mode
     sampler = ClockSampler(local)
     total_ms, per_ms, pairs, clocks = timed(args.beta, 0, sampler)
-    dense_ms, dense_per, dense_pairs, _ = timed(-math.inf, sa.FLAG_SELECT_ALL)
+    if args.no_dense:
+        dense_ms, dense_pairs = float("nan"), B * H * N * N
+    else:
+        dense_ms, dense_per, dense_pairs, _ = timed(-math.inf, sa.FLAG_SELECT_ALL)
     flops_step = sa.executed_flops(pairs, B, H, L, d, approx=True)
     fused_flops = flops_step  # the fused kernel executes all exact, proxy and routing FLOPs
     step_ms = max_over_ranks(total_ms / args.steps, pg)
@@ -349,9 +353,10 @@ def main():
         "pct_bf16_peak": 100.0 * value / world / peak,
         "stage_ms": {"pool": per_ms[0], "threshold": per_ms[1], "fused": per_ms[2]},
         "density": pairs / (B * H * N * N),
-        "dense_ms_per_call": dense_step_ms,
-        "dense_tflops": sa.executed_flops(dense_pairs, B, H, L, d, approx=False) / (dense_step_ms * 1e-3) / 1e12,
-        "speedup_vs_dense": dense_step_ms / step_ms,
+        "dense_ms_per_call": None if args.no_dense else dense_step_ms,
+        "dense_tflops": None if args.no_dense else
+        sa.executed_flops(dense_pairs, B, H, L, d, approx=False) / (dense_step_ms * 1e-3) / 1e12,
+        "speedup_vs_dense": None if args.no_dense else dense_step_ms / step_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": load_traffic(),
                      "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"

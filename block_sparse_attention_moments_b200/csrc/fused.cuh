@@ -15,21 +15,31 @@
 // blocks reach that half through the approximation instead).  The result is
 // the same as processing the blocks one by one.
 //
-// For each chunk t of C pooled keys (outer loop):
-//   route   ŝ_ij = Q̄_i·K̄_j/sqrt(d) in fp32 on CUDA cores, compared with τ_i;
-//           a warp ballot turns 32 tests into one mask word (both halves).
-//   approx  A = Q·K̄^(t)ᵀ (tcgen05, 128 x W, fp32 in TMEM, K̄ as a bf16 hi/lo
-//           pair so the logits keep K̄ to ~16 bits); per row and per
-//           column not selected by the row's half: running max m, running sum
-//           l += n_j 2^(a-m), and O += 2^(a-m) V̂_j (tcgen05, P from smem).
-//   exact   for the selected blocks of the chunk, two at a time: S = Q·[K_a;K_b]ᵀ
-//           (128 x 128), mask per half and for keys >= L, online-softmax update,
+// For each chunk t of C pooled keys (outer loop) the item's tile sequence is
+//   approx  A = Q·K̄^(t)ᵀ (128 x W, W = 32 or 64 pooled keys; K̄ as a bf16 hi/lo
+//           pair so the logits keep K̄ to ~16 bits); per row, columns not
+//           selected by the row's half get p = n_j 2^(a-m) (n_j folded into the
+//           logit as + log2 n_j), l += p and O += p V̄_j with V̄_j = V̂_j / n_j,
+//           which is Eq. 9-10's n_j e^a in the denominator and e^a V̂_j above;
+//   exact   the selected blocks of the chunk, two per tile: S = Q·[K_a;K_b]ᵀ
+//           (128 x 128), per-half / key >= L masks, online-softmax update,
 //           O += P·[V_a;V_b].
-// Epilogue: O / l in bf16 for rows < L; per-row counts |S_i|.
+// Epilogue: O / l in bf16 for rows < L.
 //
-// Shared memory (1024-byte aligned, 128-byte swizzled K-major tiles):
-//   Q 128 x d | K-side 128 x d | V-side 128 x d | P 128 x 128 | control block.
-// TMEM: columns [0, 128) hold O (fp32, lane = row), [128, 256) hold S / A.
+// Warp roles (256 threads, one persistent CTA per SM, atomic work counter):
+//   warps 0-3  softmax: one thread per tile row; masks, lazy-rescaled online
+//              softmax, P to shared memory, O correction in TMEM, epilogue.
+//   warp 4     producer of Q and of the K side (K blocks, or K̄ hi/lo) by TMA.
+//   warp 5     tcgen05 MMA issuer: S(t+1) is issued before PV(t).
+//   warp 6     producer of the V side (V blocks, or V̂) by TMA.
+//   warp 7     routing: fetches the next item, computes ŝ_ij = Q̄_i·K̄_j/sqrt(d)
+//              in fp32 for both halves, compares with τ_i (warp ballot -> mask
+//              words), one item ahead of the others (double-buffered slots).
+// Every role walks the same tile sequence, derived from the item's masks.
+//
+// Shared memory (1024-byte aligned, 128-byte swizzled tiles):
+//   Q 32 KB | K ring 2 x 32 KB | V ring 2 x 32 KB | P 32 KB | control.
+// TMEM (512 columns): O [0,128), S buffers [128,256) and [256,384).
 #pragma once
 
 #include <cstddef>
@@ -65,63 +75,155 @@ struct FusedParams {
   unsigned long long timeout_ns;
 };
 
-struct __align__(16) FusedCtl {
-  float qbar[2][128];               // pooled queries of the pair (read as float4)
+constexpr int kStages = 2;
+
+struct __align__(16) ItemSlot {
   uint32_t mask[2][kMaxMaskWords];  // selection bits of both halves
-  uint64_t bar_q;
-  uint64_t bar_kv;
-  uint64_t bar_mma;
+  int item;                         // work item index, or -1 = no more work
+  int pad[3];
+};
+
+struct __align__(16) FusedCtl {
+  ItemSlot slot[2];
+  float qbar[2][128];               // routing: pooled queries of the pair
+  uint64_t item_full[2], item_empty[2];
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full, o_done;
   uint32_t tmem_base;
-  int item;
   int abort;
-  int cnt[2];
 };
 static_assert(offsetof(FusedCtl, qbar) % 16 == 0, "float4 access to qbar");
-static_assert(offsetof(FusedCtl, bar_q) % 8 == 0, "mbarrier alignment");
+static_assert(offsetof(FusedCtl, item_full) % 8 == 0, "mbarrier alignment");
 
-constexpr uint32_t kTileBytes = 32768;  // 128 rows x 128 bf16
-constexpr uint32_t kSmemQ = 0, kSmemK = 32768, kSmemV = 65536, kSmemP = 98304, kSmemCtl = 131072;
+constexpr uint32_t kTile = 32768;  // 128 rows x 128 bf16
+constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemK = kSmemQ + kTile;
+constexpr uint32_t kSmemV = kSmemK + kStages * kTile;
+constexpr uint32_t kSmemP = kSmemV + kStages * kTile;
+constexpr uint32_t kSmemCtl = kSmemP + kTile;
 constexpr uint32_t kFusedSmemBytes = kSmemCtl + sizeof(FusedCtl) + 1024;  // + alignment slack
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemO = 0, kTmemS = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 0, kTmemS0 = 128;
+constexpr int kThreads = 256;
+constexpr int kSoftmaxThreads = 128;
+constexpr uint32_t kItemEmptyCount = kSoftmaxThreads + 3;  // softmax rows + K producer + V producer + MMA
 
 __device__ __forceinline__ bool mask_bit(const uint32_t* m, int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
 
-// First j in [from, hi) selected by either half, or hi.
-__device__ __forceinline__ int next_union(const FusedCtl& ctl, int from, int hi) {
-  int j = from;
-  while (j < hi) {
-    const int w = j >> 5;
-    const uint32_t u = (ctl.mask[0][w] | ctl.mask[1][w]) & (0xFFFFFFFFu << (j & 31));
-    if (u) {
-      const int jj = (w << 5) + __ffs(u) - 1;
-      return jj < hi ? jj : hi;
-    }
-    j = (w + 1) << 5;
-  }
-  return hi;
+// 32 selection bits starting at block j0 (bits past nw words read as 0).
+__device__ __forceinline__ uint32_t mask_bits32(const uint32_t* m, int j0, int nw) {
+  const int w = j0 >> 5, sh = j0 & 31;
+  uint32_t r = (w < nw) ? (m[w] >> sh) : 0u;
+  if (sh && w + 1 < nw) r |= m[w + 1] << (32 - sh);
+  return r;
 }
 
-// Write one row's 32 probabilities (columns [c0, c0+32)) as bf16 into the
-// 128B-swizzled K-major P tile.
-__device__ __forceinline__ void store_p32(uint8_t* sP, int row, int c0, const float (&p)[32]) {
+struct Tile {
+  int kind;    // 0 approximation, 1 exact
+  int ja, jb;  // approx: first pooled key; exact: the one or two key blocks (jb = -1: one)
+  int ncols;   // MMA N of S / K of PV
+  int avalid;  // approx: valid columns (rest of the tile belongs to no chunk)
+  bool first;  // first tile of its item (PV overwrites O)
+};
+
+// Walks an item's tile sequence: for each chunk, approximation sub-tiles
+// (skipped when both halves selected every block in them), then the union of
+// the selected blocks, two per tile.  Every warp role runs its own copy.
+struct TileIter {
+  const uint32_t* m0;
+  const uint32_t* m1;
+  int N, C, W, nw;
+  bool has1, exact_only, first;
+  int lo, hi, a0, j;
+
+  __device__ __forceinline__ int next_union(int from, int lim) const {
+    int x = from;
+    while (x < lim) {
+      const int w = x >> 5;
+      const uint32_t u = (m0[w] | m1[w]) & (0xFFFFFFFFu << (x & 31));
+      if (u) {
+        const int jj = (w << 5) + __ffs(u) - 1;
+        return jj < lim ? jj : lim;
+      }
+      x = (w + 1) << 5;
+    }
+    return lim;
+  }
+  __device__ __forceinline__ void start_chunk() {
+    hi = min(lo + C, N);
+    a0 = exact_only ? hi : lo;
+    j = next_union(lo, hi);
+  }
+  __device__ __forceinline__ void init(const ItemSlot& s, int N_, int C_, int W_, bool has1_, bool exact_only_) {
+    m0 = s.mask[0];
+    m1 = s.mask[1];
+    N = N_;
+    C = C_;
+    W = W_;
+    nw = (N_ + 31) >> 5;
+    has1 = has1_;
+    exact_only = exact_only_;
+    first = true;
+    lo = 0;
+    start_chunk();
+  }
+  __device__ __forceinline__ bool next(Tile& t) {
+    while (lo < N) {
+      while (a0 < hi) {
+        const int a1 = min(a0 + W, hi);
+        const int s = a0;
+        a0 = a1;
+        bool any = false;
+        for (int x = s; x < a1 && !any; x += 32) {
+          const int n = min(32, a1 - x);
+          const uint32_t range = (n >= 32) ? 0xFFFFFFFFu : ((1u << n) - 1u);
+          uint32_t unsel = ~mask_bits32(m0, x, nw);
+          if (has1) unsel |= ~mask_bits32(m1, x, nw);
+          any = (unsel & range) != 0u;
+        }
+        if (any) {
+          t = Tile{0, s, -1, W, a1 - s, first};
+          first = false;
+          return true;
+        }
+      }
+      if (j < hi) {
+        const int jb = next_union(j + 1, hi);
+        if (jb < hi) {
+          t = Tile{1, j, jb, 128, 0, first};
+          j = next_union(jb + 1, hi);
+        } else {
+          t = Tile{1, j, -1, 64, 0, first};
+          j = hi;
+        }
+        first = false;
+        return true;
+      }
+      lo = hi;
+      if (lo < N) start_chunk();
+    }
+    return false;
+  }
+};
+
+// Write one row's 32 probabilities (columns [c0, c0+32)), already packed as
+// bf16 pairs, into the 128B-swizzled K-major P tile.
+__device__ __forceinline__ void store_p32(uint8_t* sP, int row, int c0, const uint32_t* pk) {
 #pragma unroll
   for (int g = 0; g < 4; ++g) {  // four 16-byte chunks of 8 columns
     const int c = c0 + 8 * g;
     const int cb = c >> 6;                      // 64-column block
     const int chunk = (c & 63) >> 3;            // 16-byte chunk within the 128-byte row
     const uint32_t off = cb * 16384u + row * 128u + (((chunk ^ (row & 7)) & 7) << 4);
-    uint4 v;
-    v.x = pack_bf16x2(p[8 * g + 0], p[8 * g + 1]);
-    v.y = pack_bf16x2(p[8 * g + 2], p[8 * g + 3]);
-    v.z = pack_bf16x2(p[8 * g + 4], p[8 * g + 5]);
-    v.w = pack_bf16x2(p[8 * g + 6], p[8 * g + 7]);
-    *reinterpret_cast<uint4*>(sP + off) = v;
+    *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     sol_attn_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
                           const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_vb,
@@ -137,21 +239,28 @@ __global__ void __launch_bounds__(128, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int KSTEPS = D / 16;           // MMA K-steps over the head dimension
   constexpr uint32_t CB = 16384;           // bytes per 64-column block of a 128-row tile
-  const int NW = (p.N + 31) >> 5;
   volatile int* abort_flag = &ctl.abort;
+  const bool exact_only = (p.flags & kFlagExactOnly) != 0;
 
   if (tid == 0) {
-    mbar_init(&ctl.bar_q, 1);
-    mbar_init(&ctl.bar_kv, 1);
-    mbar_init(&ctl.bar_mma, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctl.item_full[s], 1);
+      mbar_init(&ctl.item_empty[s], kItemEmptyCount);
+      mbar_init(&ctl.s_full[s], 1);
+      mbar_init(&ctl.s_empty[s], kSoftmaxThreads);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctl.k_full[s], 1);
+      mbar_init(&ctl.k_empty[s], 1);
+      mbar_init(&ctl.v_full[s], 1);
+      mbar_init(&ctl.v_empty[s], 1);
+    }
+    mbar_init(&ctl.q_full, 1);
+    mbar_init(&ctl.q_empty, 1);
+    mbar_init(&ctl.p_full, kSoftmaxThreads);
+    mbar_init(&ctl.o_done, 1);
     ctl.abort = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_kb);
-    tma_prefetch_desc(&tm_kl);
-    tma_prefetch_desc(&tm_vb);
   }
   if (warp == 0) {
     tmem_alloc(&ctl.tmem_base, kTmemCols);
@@ -161,298 +270,416 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl.tmem_base;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tO = tmem + kTmemO + lane_base;
-  const uint32_t tS = tmem + kTmemS + lane_base;
 
-  uint32_t ph_q = 0, ph_kv = 0, ph_mma = 0;
-  const uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
-  const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
-  const int row = tid;                     // this thread's row of the 128-row tile
-  const int half = row >> 6;
-  const int tail_n = p.L - 64 * (p.N - 1);
-
-  // Wait for one mbarrier phase.  On a timeout the thread raises the CTA's
-  // abort flag and the status word; from then on every wait returns at once,
-  // thread 0 issues no more copies or MMAs, and all threads run the same
-  // (now empty) control flow to the end of the item, so no barrier is missed.
-  auto wait_all = [&](uint64_t* bar, uint32_t& ph) {
-    const bool ok = mbar_wait(bar, ph, abort_flag, p.timeout_ns);
-    ph ^= 1u;
-    if (!ok) {
-      *abort_flag = 1;
-      atomicOr(p.status, kStatusTimeout);
-    }
+  // Bounded wait; on a timeout raise the abort flag and the status word.  All
+  // later waits return false at once, every role leaves its loop, and the CTA
+  // meets at the final barrier.
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (mbar_wait(bar, parity, abort_flag, p.timeout_ns)) return true;
+    *abort_flag = 1;
+    atomicOr(p.status, kStatusTimeout);
+    return false;
   };
-  auto issuer = [&]() -> bool { return tid == 0 && *abort_flag == 0; };
 
-  for (;;) {
-    if (tid == 0) ctl.item = *abort_flag ? p.num_items : static_cast<int>(atomicAdd(p.work_counter, 1u));
-    __syncthreads();
-    const int item = ctl.item;
-    if (item >= p.num_items) break;
-    const int bh = item / p.num_pairs;
-    const int pair = item - bh * p.num_pairs;
-    const int i0 = 2 * pair, i1 = 2 * pair + 1;
-    const bool has1 = i1 < p.N;
-
-    // ---- load the 128-row query tile (TMA, zero-filled past L)
-    if (issuer()) {
-      mbar_arrive_expect_tx(&ctl.bar_q, 128u * D * 2u);
-#pragma unroll
-      for (int cb = 0; cb < D / 64; ++cb) tma_load_3d(sQ + cb * CB, &tm_q, &ctl.bar_q, cb * 64, 128 * pair, bh);
-    }
-
-    // ---- routing for the whole pair (method: Eq. 6-7; tested as ŝ >= τ)
-    const float* qb = p.qbar + static_cast<size_t>(bh) * p.N * D;
-    const float* kb = p.kbar + static_cast<size_t>(bh) * p.N * D;
-    for (int e = tid; e < 2 * D; e += 128) {
-      const int h = e / D, c = e % D;
-      const int i = h ? i1 : i0;
-      ctl.qbar[h][c] = (i < p.N) ? qb[static_cast<size_t>(i) * D + c] : 0.f;
-    }
-    if (tid < 2) ctl.cnt[tid] = 0;
-    __syncthreads();
-    const float tau0 = p.tau[static_cast<size_t>(bh) * p.N + i0];
-    const float tau1 = has1 ? p.tau[static_cast<size_t>(bh) * p.N + i1] : INFINITY;
-    int my_cnt0 = 0, my_cnt1 = 0;
-    for (int g = warp; g < NW; g += 4) {
-      const int j = 32 * g + lane;
-      bool s0 = false, s1 = false;
-      if (j < p.N) {
-        const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
-        float d0 = 0.f, d1 = 0.f;
-#pragma unroll 8
-        for (int c4 = 0; c4 < D / 4; ++c4) {
-          const float4 x = __ldg(kr + c4);
-          const float4 a = *reinterpret_cast<const float4*>(&ctl.qbar[0][4 * c4]);
-          const float4 b = *reinterpret_cast<const float4*>(&ctl.qbar[1][4 * c4]);
-          d0 = fmaf(a.x, x.x, d0); d0 = fmaf(a.y, x.y, d0); d0 = fmaf(a.z, x.z, d0); d0 = fmaf(a.w, x.w, d0);
-          d1 = fmaf(b.x, x.x, d1); d1 = fmaf(b.y, x.y, d1); d1 = fmaf(b.z, x.z, d1); d1 = fmaf(b.w, x.w, d1);
+  if (warp == 7) {
+    // =========================================================== routing
+    for (int seq = 0;; ++seq) {
+      const int s = seq & 1;
+      if (seq >= 2 && !wait(&ctl.item_empty[s], ((seq >> 1) - 1) & 1)) break;
+      int item = 0;
+      if (lane == 0) item = static_cast<int>(atomicAdd(p.work_counter, 1u));
+      item = __shfl_sync(0xFFFFFFFFu, item, 0);
+      ItemSlot& sl = ctl.slot[s];
+      if (item >= p.num_items) {
+        if (lane == 0) {
+          sl.item = -1;
+          mbar_arrive(&ctl.item_full[s]);
         }
-        s0 = d0 * p.inv_sqrt_d >= tau0;
-        s1 = has1 && (d1 * p.inv_sqrt_d >= tau1);
+        break;
       }
-      const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, s0);
-      const uint32_t m1 = __ballot_sync(0xFFFFFFFFu, s1);
-      if (lane == 0) {
-        ctl.mask[0][g] = m0;
-        ctl.mask[1][g] = m1;
-        my_cnt0 += __popc(m0);
-        my_cnt1 += __popc(m1);
-      }
-    }
-    if (lane == 0) {
-      atomicAdd(&ctl.cnt[0], my_cnt0);
-      atomicAdd(&ctl.cnt[1], my_cnt1);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      p.counts[static_cast<size_t>(bh) * p.N + i0] = ctl.cnt[0];
-      if (has1) p.counts[static_cast<size_t>(bh) * p.N + i1] = ctl.cnt[1];
-    }
-    if (p.mask_out) {
-      for (int e = tid; e < 2 * NW; e += 128) {
-        const int h = e / NW, g = e % NW;
+      const int bh = item / p.num_pairs;
+      const int pair = item - bh * p.num_pairs;
+      const int i0 = 2 * pair, i1 = 2 * pair + 1;
+      const bool has1 = i1 < p.N;
+      const float* qb = p.qbar + static_cast<size_t>(bh) * p.N * D;
+      const float* kb = p.kbar + static_cast<size_t>(bh) * p.N * D;
+      for (int e = lane; e < 2 * D; e += 32) {
+        const int h = e / D, c = e % D;
         const int i = h ? i1 : i0;
-        if (i < p.N) p.mask_out[(static_cast<size_t>(bh) * p.N + i) * NW + g] = ctl.mask[h][g];
+        ctl.qbar[h][c] = (i < p.N) ? qb[static_cast<size_t>(i) * D + c] : 0.f;
+      }
+      __syncwarp();
+      const float tau0 = p.tau[static_cast<size_t>(bh) * p.N + i0];
+      const float tau1 = has1 ? p.tau[static_cast<size_t>(bh) * p.N + i1] : INFINITY;
+      const int NW = (p.N + 31) >> 5;
+      int cnt0 = 0, cnt1 = 0;
+      for (int g = 0; g < NW; ++g) {
+        const int j = 32 * g + lane;
+        bool s0 = false, s1 = false;
+        if (j < p.N) {
+          const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
+#pragma unroll 8
+          for (int c4 = 0; c4 < D / 4; ++c4) {
+            const float4 x = __ldg(kr + c4);
+            const float4 qa = *reinterpret_cast<const float4*>(&ctl.qbar[0][4 * c4]);
+            const float4 qb4 = *reinterpret_cast<const float4*>(&ctl.qbar[1][4 * c4]);
+            a0 = fmaf(qa.x, x.x, a0); a1 = fmaf(qa.y, x.y, a1); a2 = fmaf(qa.z, x.z, a2); a3 = fmaf(qa.w, x.w, a3);
+            b0 = fmaf(qb4.x, x.x, b0); b1 = fmaf(qb4.y, x.y, b1); b2 = fmaf(qb4.z, x.z, b2); b3 = fmaf(qb4.w, x.w, b3);
+          }
+          const float d0 = (a0 + a1) + (a2 + a3);
+          const float d1 = (b0 + b1) + (b2 + b3);
+          s0 = d0 * p.inv_sqrt_d >= tau0;
+          s1 = has1 && (d1 * p.inv_sqrt_d >= tau1);
+        }
+        const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, s0);
+        const uint32_t m1 = __ballot_sync(0xFFFFFFFFu, s1);
+        if (lane == 0) {
+          sl.mask[0][g] = m0;
+          sl.mask[1][g] = m1;
+        }
+        cnt0 += __popc(m0);
+        cnt1 += __popc(m1);
+      }
+      if (lane == 0) {
+        p.counts[static_cast<size_t>(bh) * p.N + i0] = cnt0;
+        if (has1) p.counts[static_cast<size_t>(bh) * p.N + i1] = cnt1;
+        sl.item = item;
+      }
+      __syncwarp();
+      if (p.mask_out) {
+        for (int e = lane; e < 2 * NW; e += 32) {
+          const int h = e / NW, g = e % NW;
+          const int i = h ? i1 : i0;
+          if (i < p.N) p.mask_out[(static_cast<size_t>(bh) * p.N + i) * NW + g] = sl.mask[h][g];
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.item_full[s]);   // release: masks and item visible
+    }
+  } else if (warp == 4 || warp == 6) {
+    // =========================================================== TMA producers
+    const bool kside = (warp == 4);
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int seq = 0;; ++seq) {
+        const int s = seq & 1;
+        if (!wait(&ctl.item_full[s], (seq >> 1) & 1)) break;
+        const ItemSlot& sl = ctl.slot[s];
+        const int item = sl.item;
+        if (item < 0) break;
+        const int bh = item / p.num_pairs;
+        const int pair = item - bh * p.num_pairs;
+        bool ok = true;
+        if (kside) {  // query tile of the item (the previous item's S MMAs must be done)
+          if (seq > 0 && !wait(&ctl.q_empty, (seq - 1) & 1)) break;
+          mbar_arrive_expect_tx(&ctl.q_full, 128u * D * 2u);
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_3d(sQ + cb * CB, &tm_q, &ctl.q_full, cb * 64, 128 * pair, bh);
+        }
+        TileIter it;
+        it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
+        Tile t;
+        while (it.next(t)) {
+          uint64_t* empty = kside ? &ctl.k_empty[stage] : &ctl.v_empty[stage];
+          uint64_t* full = kside ? &ctl.k_full[stage] : &ctl.v_full[stage];
+          if (!wait(empty, phase ^ 1u)) { ok = false; break; }
+          uint8_t* dst = (kside ? sK : sV) + stage * kTile;
+          if (t.kind == 0) {
+            mbar_arrive_expect_tx(full, (kside ? 2u : 1u) * p.W * D * 2u);
+#pragma unroll
+            for (int cb = 0; cb < D / 64; ++cb) {
+              if (kside) {
+                tma_load_3d(dst + cb * CB, &tm_kb, full, cb * 64, t.ja, bh);
+                tma_load_3d(dst + cb * CB + 8192, &tm_kl, full, cb * 64, t.ja, bh);
+              } else {
+                tma_load_3d(dst + cb * CB, &tm_vb, full, cb * 64, t.ja, bh);
+              }
+            }
+          } else {
+            const int nblk = (t.jb >= 0) ? 2 : 1;
+            mbar_arrive_expect_tx(full, static_cast<uint32_t>(nblk) * 64u * D * 2u);
+            const CUtensorMap* map = kside ? &tm_k : &tm_v;
+#pragma unroll
+            for (int cb = 0; cb < D / 64; ++cb) {
+              tma_load_3d(dst + cb * CB, map, full, cb * 64, 64 * t.ja, bh);
+              if (nblk == 2) tma_load_3d(dst + cb * CB + 8192, map, full, cb * 64, 64 * t.jb, bh);
+            }
+          }
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        mbar_arrive(&ctl.item_empty[s]);
+        if (!ok) break;
       }
     }
-
-    // ---- online-softmax state of this thread's row (log2 domain)
-    float m_run = -INFINITY, l_run = 0.f;
-    bool o_init = false;
-    wait_all(&ctl.bar_q, ph_q);
-
-    const uint32_t* own = ctl.mask[half];
-    const bool exact_only = (p.flags & kFlagExactOnly) != 0;
-
-    // One tile: issue S MMA (tid 0), online-softmax on this thread's row,
-    // issue PV MMA.  kind 0 = approximation, 1 = exact.
-    auto process_tile = [&](int kind, int ncols_mma, int ja, int jb, int a_valid) {
-      // S / A = Q · Kside^T
-      if (issuer()) {
+  } else if (warp == 5) {
+    // =========================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
+      int kstage = 0, vstage = 0;
+      uint32_t kphase = 0, vphase = 0;
+      uint32_t tcount = 0;   // tiles whose S MMA is issued (S buffer = index & 1)
+      bool pend = false;     // the PV of tile pv_idx is still to be issued
+      Tile pt{};
+      uint32_t pv_idx = 0;
+      int pv_stage = 0;
+      uint32_t pv_phase = 0;
+      bool ok = true;
+      // O (+)= P · Vside for the pending tile.
+      auto issue_pv = [&]() -> bool {
+        if (!wait(&ctl.p_full, pv_idx & 1)) return false;
+        if (!wait(&ctl.v_full[pv_stage], pv_phase)) return false;
         tc_fence_after();
-        const uint32_t idesc_s = idesc_bf16_f32(128, ncols_mma, 0);
-#pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-          const uint32_t koff = (kk >> 2) * CB + (kk & 3) * 32;
-          umma_ss(tmem + kTmemS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(sKa + koff, 16, 1024), idesc_s,
-                  kk > 0 ? 1u : 0u);
+        const int ksteps = pt.ncols / 16;
+        const uint32_t vbase = sVa + pv_stage * kTile;
+        for (int kk = 0; kk < ksteps; ++kk) {
+          const uint32_t poff = (kk >> 2) * CB + (kk & 3) * 32;
+          umma_ss(tmem + kTmemO, sdesc_sw128(sPa + poff, 16, 1024), sdesc_sw128(vbase + kk * 2048, CB, 1024),
+                  idesc_pv, (pt.first && kk == 0) ? 0u : 1u);
         }
-        if (kind == 0) {  // + Q · K̄_lo^T (rows 64.. of the K-side tile)
+        umma_commit(&ctl.o_done);
+        umma_commit(&ctl.v_empty[pv_stage]);
+        pend = false;
+        return true;
+      };
+      for (int seq = 0;; ++seq) {
+        const int s = seq & 1;
+        if (!wait(&ctl.item_full[s], (seq >> 1) & 1)) { ok = false; break; }
+        const ItemSlot& sl = ctl.slot[s];
+        const int item = sl.item;
+        if (item < 0) break;
+        const int pair = item % p.num_pairs;
+        if (!wait(&ctl.q_full, seq & 1)) { ok = false; break; }
+        TileIter it;
+        it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
+        Tile t;
+        while (it.next(t)) {
+          // S(t) = Q · Kside^T into S buffer (tcount & 1)
+          const int b = tcount & 1;
+          if (tcount >= 2 && !wait(&ctl.s_empty[b], ((tcount >> 1) - 1) & 1)) { ok = false; break; }
+          if (!wait(&ctl.k_full[kstage], kphase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t dS = tmem + kTmemS0 + b * 128;
+          const uint32_t kbase = sKa + kstage * kTile;
+          const uint32_t idesc_s = idesc_bf16_f32(128, t.ncols, 0);
 #pragma unroll
           for (int kk = 0; kk < KSTEPS; ++kk) {
             const uint32_t koff = (kk >> 2) * CB + (kk & 3) * 32;
-            umma_ss(tmem + kTmemS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(sKa + 8192 + koff, 16, 1024),
-                    idesc_s, 1u);
+            umma_ss(dS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(kbase + koff, 16, 1024), idesc_s,
+                    kk > 0 ? 1u : 0u);
           }
-        }
-        umma_commit(&ctl.bar_mma);
-      }
-      wait_all(&ctl.bar_mma, ph_mma);
-      tc_fence_after();
-
-      // masked logits of this row
-      float x[128];
+          if (t.kind == 0) {  // + Q · K̄_lo^T (rows 64.. of the K-side tile)
 #pragma unroll
-      for (int c32 = 0; c32 < 4; ++c32) {
-        if (c32 * 32 < ncols_mma) {
-          uint32_t r[32];
-          tmem_ld_x32(tS + c32 * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[c32 * 32 + e] = __uint_as_float(r[e]) * p.scale_log2;
-        }
-      }
-      // validity bitmap of the row's columns: vm[c32] bit e <-> column 32*c32 + e
-      uint32_t vm[4];
-#pragma unroll
-      for (int c32 = 0; c32 < 4; ++c32) {
-        uint32_t bits = 0u;
-        if (c32 * 32 < ncols_mma) {
-          if (kind == 0) {
-            const int c0 = 32 * c32;
-            const int nv = min(max(a_valid - c0, 0), 32);
-            const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
-            const int j0 = ja + c0;
-            const int w = j0 >> 5, sh = j0 & 31;
-            uint32_t sel = (w < NW) ? (own[w] >> sh) : 0u;
-            if (sh && w + 1 < NW) sel |= own[w + 1] << (32 - sh);
-            bits = range & ~sel;
-          } else {
-            const int jx = (c32 < 2) ? ja : jb;
-            const int key0 = 64 * jx + 32 * (c32 & 1);
-            const int nv = min(max(p.L - key0, 0), 32);
-            const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
-            bits = mask_bit(own, jx) ? range : 0u;
-          }
-        }
-        vm[c32] = bits;
-      }
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if ((vm[c >> 5] >> (c & 31)) & 1u) tmax = fmaxf(tmax, x[c]);
-      // lazy rescale: move the reference max only when it grows by > 8 (x256).
-      // TMEM loads/stores are warp-collective, so the O update runs for the
-      // whole warp when any of its rows needs it (alpha = 1 for the others).
-      const bool need = tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY);
-      float alpha = 1.f;
-      if (need) {
-        const float m_new = fmaxf(m_run, tmax);
-        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
-        l_run *= alpha;
-        m_run = m_new;
-      }
-      if (o_init && __any_sync(0xFFFFFFFFu, need)) {
-#pragma unroll
-        for (int c32 = 0; c32 < D / 32; ++c32) {
-          uint32_t r[32];
-          tmem_ld_x32(tO + c32 * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st_x32(tO + c32 * 32, r);
-        }
-        tmem_st_wait();
-      }
-      const float m_ref = (m_run == -INFINITY) ? 0.f : m_run;
-      // tail block weight for the approximation (n_j of the ragged last block)
-      const int tail_col = (kind == 0) ? (p.N - 1 - ja) : -1;
-      float ps = 0.f;
-#pragma unroll
-      for (int c32 = 0; c32 < 4; ++c32) {
-        if (c32 * 32 < ncols_mma) {
-          float pr[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = c32 * 32 + e;
-            const bool valid = (vm[c32] >> e) & 1u;
-            const float pv = valid ? ex2_approx(x[c] - m_ref) : 0.f;
-            const float w = (kind == 0) ? ((c == tail_col) ? static_cast<float>(tail_n) : 64.f) : 1.f;
-            ps = fmaf(w, pv, ps);
-            pr[e] = pv;
-          }
-          store_p32(sP, row, c32 * 32, pr);
-        }
-      }
-      l_run += ps;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      // O += P · Vside
-      if (issuer()) {
-        tc_fence_after();
-        const int ksteps = ncols_mma / 16;
-        for (int kk = 0; kk < ksteps; ++kk) {
-          const uint32_t poff = (kk >> 2) * CB + (kk & 3) * 32;
-          umma_ss(tmem + kTmemO, sdesc_sw128(sPa + poff, 16, 1024), sdesc_sw128(sVa + kk * 2048, CB, 1024),
-                  idesc_pv, (o_init || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&ctl.bar_mma);
-      }
-      wait_all(&ctl.bar_mma, ph_mma);
-      tc_fence_after();
-      o_init = true;
-    };
-
-    const int C = p.chunk;
-    for (int lo = 0; lo < p.N; lo += C) {
-      const int hi = min(lo + C, p.N);
-      // -- approximation sub-tiles of this chunk (Eq. 9-11)
-      if (!exact_only) {
-        for (int a0 = lo; a0 < hi; a0 += p.W) {
-          const int a1 = min(a0 + p.W, hi);
-          // skip when every column is selected by both halves (nothing to approximate)
-          bool any = false;
-          for (int j = a0; j < a1 && !any; ++j)
-            any = !mask_bit(ctl.mask[0], j) || (has1 && !mask_bit(ctl.mask[1], j));
-          if (!any) continue;
-          if (issuer()) {
-            mbar_arrive_expect_tx(&ctl.bar_kv, 3u * p.W * D * 2u);
-#pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb) {
-              tma_load_3d(sK + cb * CB, &tm_kb, &ctl.bar_kv, cb * 64, a0, bh);
-              tma_load_3d(sK + cb * CB + 8192, &tm_kl, &ctl.bar_kv, cb * 64, a0, bh);
-              tma_load_3d(sV + cb * CB, &tm_vb, &ctl.bar_kv, cb * 64, a0, bh);
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+              const uint32_t koff = (kk >> 2) * CB + (kk & 3) * 32;
+              umma_ss(dS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(kbase + 8192 + koff, 16, 1024),
+                      idesc_s, 1u);
             }
           }
-          wait_all(&ctl.bar_kv, ph_kv);
-          process_tile(0, p.W, a0, 0, a1 - a0);
-        }
-      }
-      // -- exact inner loop over the selected blocks of this chunk (Eq. 7)
-      int j = next_union(ctl, lo, hi);
-      while (j < hi) {
-        const int jb = next_union(ctl, j + 1, hi);
-        const int nblk = (jb < hi) ? 2 : 1;
-        if (issuer()) {
-          mbar_arrive_expect_tx(&ctl.bar_kv, static_cast<uint32_t>(nblk) * 2u * 64u * D * 2u);
-#pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb) {
-            tma_load_3d(sK + cb * CB, &tm_k, &ctl.bar_kv, cb * 64, 64 * j, bh);
-            tma_load_3d(sV + cb * CB, &tm_v, &ctl.bar_kv, cb * 64, 64 * j, bh);
-            if (nblk == 2) {
-              tma_load_3d(sK + cb * CB + 8192, &tm_k, &ctl.bar_kv, cb * 64, 64 * jb, bh);
-              tma_load_3d(sV + cb * CB + 8192, &tm_v, &ctl.bar_kv, cb * 64, 64 * jb, bh);
-            }
+          umma_commit(&ctl.s_full[b]);
+          umma_commit(&ctl.k_empty[kstage]);
+          if (++kstage == kStages) {
+            kstage = 0;
+            kphase ^= 1u;
           }
+          // PV of the previous tile, now that S(t) is queued ahead of it
+          if (pend && !issue_pv()) { ok = false; break; }
+          pt = t;
+          pend = true;
+          pv_idx = tcount;
+          pv_stage = vstage;
+          pv_phase = vphase;
+          if (++vstage == kStages) {
+            vstage = 0;
+            vphase ^= 1u;
+          }
+          ++tcount;
         }
-        wait_all(&ctl.bar_kv, ph_kv);
-        process_tile(1, 64 * nblk, j, nblk == 2 ? jb : -1, 0);
-        j = (nblk == 2) ? next_union(ctl, jb + 1, hi) : hi;
+        if (!ok) break;
+        // every S MMA of this item is issued: Q is free once they complete
+        umma_commit(&ctl.q_empty);
+        mbar_arrive(&ctl.item_empty[s]);
       }
+      if (ok && pend) issue_pv();
     }
-    // ---- epilogue: O / l for rows < L (Eq. 10 normalisation)
-    {
+  } else {
+    // =========================================================== softmax (warps 0-3)
+    const int row = tid;              // tile row = TMEM lane
+    const int half = row >> 6;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tO = tmem + kTmemO + lane_base;
+    const int tail_n = p.L - 64 * (p.N - 1);
+    uint32_t tcount = 0;     // tiles processed
+    uint32_t pv_seen = 0;    // PV completions waited for
+    bool ok = true;
+    for (int seq = 0; ok; ++seq) {
+      const int s = seq & 1;
+      if (!wait(&ctl.item_full[s], (seq >> 1) & 1)) break;
+      const ItemSlot& sl = ctl.slot[s];
+      const int item = sl.item;
+      if (item < 0) break;
+      const int bh = item / p.num_pairs;
+      const int pair = item - bh * p.num_pairs;
+      const uint32_t* own = sl.mask[half];
+      const int NW = (p.N + 31) >> 5;
+      float m_run = -INFINITY, l_run = 0.f;
+      bool any_tile = false;
+      TileIter it;
+      it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
+      Tile t;
+      while (it.next(t)) {
+        any_tile = true;
+        const int b = tcount & 1;
+        if (!wait(&ctl.s_full[b], (tcount >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tS = tmem + kTmemS0 + b * 128 + lane_base;
+        // Two passes over the tile in 32-column groups, each reading S from
+        // TMEM: the first finds the row maximum, the second writes P.  Keeping
+        // one group in registers at a time keeps the loop body small.
+        const int ng = t.ncols >> 5;
+        // validity of a group's 32 columns (warp-uniform: a warp's rows share a half)
+        auto group_bits = [&](int g) -> uint32_t {
+          const int c0 = 32 * g;
+          if (t.kind == 0) {
+            const int nv = min(max(t.avalid - c0, 0), 32);
+            const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+            return range & ~mask_bits32(own, t.ja + c0, NW);
+          }
+          const int jx = (g < 2) ? t.ja : t.jb;
+          const int key0 = 64 * jx + 32 * (g & 1);
+          const int nv = min(max(p.L - key0, 0), 32);
+          const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+          return mask_bit(own, jx) ? range : 0u;
+        };
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll 1
+        for (int g = 0; g < ng; ++g) {
+          float xv[32];
+          tmem_ld_x32f(tS + 32 * g, xv);
+          tmem_ld_wait();
+          reg_fence32(xv);
+          const uint32_t bits = group_bits(g);
+          if (bits != 0xFFFFFFFFu) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            mx0 = fmaxf(mx0, xv[e]);
+            mx1 = fmaxf(mx1, xv[e + 1]);
+            mx2 = fmaxf(mx2, xv[e + 2]);
+            mx3 = fmaxf(mx3, xv[e + 3]);
+          }
+        }
+        const float rmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        // In log2 units.  An approximation column stands for its n_j tokens:
+        // its weight n_j is folded into the logit as + log2(n_j) (6 for a full
+        // block) and the value side uses the block mean V̂_j / n_j.
+        const float boost = (t.kind == 0) ? 6.f : 0.f;
+        const float tmax = (rmax == -INFINITY) ? -INFINITY : fmaf(rmax, p.scale_log2, boost);
+        // lazy rescale: move the reference max only when it grows by > 8 (x256)
+        const bool need = tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY);
+        float alpha = 1.f;
+        if (need) {
+          const float m_new = fmaxf(m_run, tmax);
+          alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        const float off = boost - ((m_run == -INFINITY) ? 0.f : m_run);
+        // the ragged last block, when it is an approximation column, weighs tail_n
+        const int tail_col = (t.kind == 0 && tail_n != 64) ? (p.N - 1 - t.ja) : -1;
+        const int tail_g = (tail_col >= 0 && tail_col < t.ncols) ? (tail_col >> 5) : -1;
+        const float off_tail = off + (log2f(static_cast<float>(tail_n)) - 6.f);
+        // the previous tile's PV must be done before P is overwritten or O rescaled
+        if (pv_seen < tcount) {
+          if (!wait(&ctl.o_done, (tcount - 1) & 1)) { ok = false; break; }
+          pv_seen = tcount;
+          tc_fence_after();
+        }
+        if (!t.first && __any_sync(0xFFFFFFFFu, need)) {
+#pragma unroll 1
+          for (int c32 = 0; c32 < D / 32; ++c32) {
+            uint32_t r[32];
+            tmem_ld_x32(tO + c32 * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st_x32(tO + c32 * 32, r);
+          }
+          tmem_st_wait();
+        }
+        float sm0 = 0.f, sm1 = 0.f, sm2 = 0.f, sm3 = 0.f;
+#pragma unroll 1
+        for (int g = 0; g < ng; ++g) {
+          float xv[32];
+          tmem_ld_x32f(tS + 32 * g, xv);
+          tmem_ld_wait();
+          reg_fence32(xv);
+          const uint32_t bits = group_bits(g);
+          if (bits != 0xFFFFFFFFu) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
+          }
+          uint32_t pk[16];
+          if (g != tail_g) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float p0 = ex2_approx(fmaf(xv[e], p.scale_log2, off));
+              const float p1 = ex2_approx(fmaf(xv[e + 1], p.scale_log2, off));
+              const float p2 = ex2_approx(fmaf(xv[e + 2], p.scale_log2, off));
+              const float p3 = ex2_approx(fmaf(xv[e + 3], p.scale_log2, off));
+              sm0 += p0;
+              sm1 += p1;
+              sm2 += p2;
+              sm3 += p3;
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+              pk[(e >> 1) + 1] = pack_bf16x2(p2, p3);
+            }
+          } else {
+            const int et = tail_col & 31;
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float p0 = ex2_approx(fmaf(xv[e], p.scale_log2, e == et ? off_tail : off));
+              const float p1 = ex2_approx(fmaf(xv[e + 1], p.scale_log2, e + 1 == et ? off_tail : off));
+              sm0 += p0;
+              sm1 += p1;
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
+          }
+          store_p32(sP, row, 32 * g, pk);
+        }
+        l_run += (sm0 + sm1) + (sm2 + sm3);
+        // S buffer b may now be overwritten by the MMA of tile tcount + 2
+        tc_fence_before();
+        mbar_arrive(&ctl.s_empty[b]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&ctl.p_full);
+        ++tcount;
+      }
+      if (!ok) break;
+      // ---- epilogue: wait for the item's last PV, O / l for rows < L (Eq. 10)
+      if (tcount > pv_seen) {
+        if (!wait(&ctl.o_done, (tcount - 1) & 1)) break;
+        pv_seen = tcount;
+        tc_fence_after();
+      }
       const int token = 128 * pair + row;
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       uint16_t* orow = p.out + (static_cast<size_t>(bh) * p.L + token) * D;
 #pragma unroll
       for (int c32 = 0; c32 < D / 32; ++c32) {
         uint32_t r[32];
-        if (o_init) {
+        if (any_tile) {            // an item with no tile (exact-only, nothing selected) outputs 0
           tmem_ld_x32(tO + c32 * 32, r);
           tmem_ld_wait();
         } else {
@@ -471,14 +698,14 @@ __global__ void __launch_bounds__(128, 1)
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&ctl.item_empty[s]);
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
   }
 
   // After a timeout, give copies or MMAs that may still be in flight a bounded
   // time to land before the shared memory and TMEM are released.
+  __syncwarp();
   if (*abort_flag) {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);

@@ -7,6 +7,10 @@
 //   V̂_j = sum of its valid values; a ragged last block is pooled over its
 //   valid tokens only.
 //
+// The fused kernel's approximation multiplies probabilities that already carry
+// the block's token count n_j by the block mean V̂_j / n_j, so V is also written
+// as that mean in bf16 (V̂ itself is only exported for checks).
+//
 // K̄ is also written as a bf16 pair (hi, lo = bf16(K̄ - hi)): the approximation
 // tile multiplies Q by both, so its logits carry K̄ to ~16 significant bits
 // rather than bf16's 8 (the exact path's K is bf16 input and needs no split).
@@ -45,7 +49,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
                                                    float* __restrict__ qbar, float* __restrict__ kbar,
                                                    __nv_bfloat16* __restrict__ kbar_bf,
                                                    __nv_bfloat16* __restrict__ kbar_lo,
-                                                   __nv_bfloat16* __restrict__ vhat_bf,
+                                                   __nv_bfloat16* __restrict__ vbar_bf,
                                                    float* __restrict__ vhat_f32 /* nullable */) {
   constexpr int TPR = D / 8;      // threads per token row (16 bytes each)
   constexpr int RPP = 256 / TPR;  // token rows per pass
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
     const __nv_bfloat16 hi = __float2bfloat16_rn(mk);
     kbar_bf[o] = hi;
     kbar_lo[o] = __float2bfloat16_rn(mk - __bfloat162float(hi));
-    vhat_bf[o] = __float2bfloat16_rn(sv);
+    vbar_bf[o] = __float2bfloat16_rn(sv / fn);
     if (vhat_f32) vhat_f32[o] = sv;
   }
 }

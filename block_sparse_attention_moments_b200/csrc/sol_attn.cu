@@ -57,7 +57,7 @@ struct Workspace {
   float* kbar = nullptr;
   __nv_bfloat16* kbar_bf = nullptr;
   __nv_bfloat16* kbar_lo = nullptr;
-  __nv_bfloat16* vhat_bf = nullptr;
+  __nv_bfloat16* vbar_bf = nullptr;
   double* mom_mean = nullptr;
   double* mom_cov = nullptr;
   float* tau = nullptr;
@@ -103,7 +103,7 @@ size_t layout(const Shape& s, Workspace* w, char* base) {
     w->kbar = reinterpret_cast<float*>(p_kbar);
     w->kbar_bf = reinterpret_cast<__nv_bfloat16*>(p_kbf);
     w->kbar_lo = reinterpret_cast<__nv_bfloat16*>(p_klo);
-    w->vhat_bf = reinterpret_cast<__nv_bfloat16*>(p_vbf);
+    w->vbar_bf = reinterpret_cast<__nv_bfloat16*>(p_vbf);
     w->mom_mean = reinterpret_cast<double*>(p_mean);
     w->mom_cov = reinterpret_cast<double*>(p_cov);
     w->tau = reinterpret_cast<float*>(p_tau);
@@ -225,10 +225,10 @@ int run_pool(Workspace& w, const void* q, const void* k, const void* v, const so
   auto kk = static_cast<const uint16_t*>(k);
   auto vv = static_cast<const uint16_t*>(v);
   if (s.d == 128)
-    pool_kernel<128><<<grid, 256, 0, st>>>(qq, kk, vv, s.L, N, w.qbar, w.kbar, w.kbar_bf, w.kbar_lo, w.vhat_bf,
+    pool_kernel<128><<<grid, 256, 0, st>>>(qq, kk, vv, s.L, N, w.qbar, w.kbar, w.kbar_bf, w.kbar_lo, w.vbar_bf,
                                            vdbg);
   else
-    pool_kernel<64><<<grid, 256, 0, st>>>(qq, kk, vv, s.L, N, w.qbar, w.kbar, w.kbar_bf, w.kbar_lo, w.vhat_bf,
+    pool_kernel<64><<<grid, 256, 0, st>>>(qq, kk, vv, s.L, N, w.qbar, w.kbar, w.kbar_bf, w.kbar_lo, w.vbar_bf,
                                           vdbg);
   CUDA_TRY(cudaGetLastError());
   const size_t nbytes = static_cast<size_t>(s.B) * s.H * N * s.d * 4;
@@ -288,7 +288,7 @@ int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void
   if ((rc = make_map(&tv, v, D, s.L, BH, 64))) return rc;
   if ((rc = make_map(&tkb, w.kbar_bf, D, N, BH, W))) return rc;
   if ((rc = make_map(&tkl, w.kbar_lo, D, N, BH, W))) return rc;
-  if ((rc = make_map(&tvb, w.vhat_bf, D, N, BH, W))) return rc;
+  if ((rc = make_map(&tvb, w.vbar_bf, D, N, BH, W))) return rc;
 
   FusedParams p{};
   p.BH = static_cast<int>(BH);
@@ -322,7 +322,7 @@ int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void
   }
   CUDA_TRY(cudaMemsetAsync(w.counter, 0, sizeof(unsigned), st));
   const int grid = std::min(p.num_items, nsm);
-  sol_attn_fused_kernel<D><<<grid, 128, kFusedSmemBytes, st>>>(tq, tk, tv, tkb, tkl, tvb, p);
+  sol_attn_fused_kernel<D><<<grid, kThreads, kFusedSmemBytes, st>>>(tq, tk, tv, tkb, tkl, tvb, p);
   CUDA_TRY(cudaGetLastError());
   return SOL_ATTN_OK;
 }
