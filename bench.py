@@ -209,6 +209,35 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_role_profile(args):
+    """Per-role cycle accounting of the fused kernel (profiling build; not a bench line)."""
+    os.environ["SOL_ATTN_PROFILE"] = "1"
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_moments_b200 as sa
+    from synth import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    qb, kb, vb = rank_inputs(wl, 0)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = dev(qb), dev(kb), dev(vb)
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    for beta, flags, tag in ((args.beta, 0, "sparse"), (-math.inf, sa.FLAG_SELECT_ALL, "dense")):
+        for _ in range(args.warmup):
+            sa.forward(q, k, v, beta, wl.chunk, flags=flags)
+        sa.profile_read(reset=True)
+        sa.forward(q, k, v, beta, wl.chunk, flags=flags)
+        prof = sa.profile_read(reset=True)
+        tiles = max(prof["softmax.tiles"], 1)
+        per_cta = {k2: v2 / nsm for k2, v2 in prof.items()}
+        print(json.dumps({"workload": wl.name, "mode": tag, "ctas": nsm, "tiles_per_cta": tiles / nsm,
+                          "cycles_per_cta": {k2: round(v2) for k2, v2 in per_cta.items()},
+                          "softmax_cycles_per_tile": {k2: round(prof[k2] / tiles, 1) for k2 in
+                                                      ("softmax.pass1", "softmax.rescale", "softmax.pass2",
+                                                       "softmax.wait_s", "softmax.wait_o",
+                                                       "softmax.wait_exchange")}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -222,7 +251,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the select-all (dense) comparison run")
+    ap.add_argument("--role-profile", action="store_true",
+                    help="run the profiling build (libsol_attn_profile.so) and print per-role cycle accounting")
     args = ap.parse_args()
+    if args.role_profile:
+        return run_role_profile(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

@@ -29,7 +29,9 @@ FLAG_SYNC_CHECK = 0x4
 BLOCK = 64
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_PKG, "libsol_attn.so")
+# SOL_ATTN_PROFILE=1 selects the build with per-role cycle accounting.
+_LIB_PATH = os.path.join(_PKG, "libsol_attn_profile.so" if os.environ.get("SOL_ATTN_PROFILE") == "1"
+                         else "libsol_attn.so")
 _lib = None
 
 # Every entry point declared in include/sol_attn.h.
@@ -37,7 +39,7 @@ EXPORTED_SYMBOLS = (
     "sol_attn_forward", "sol_attn_forward_ex", "sol_attn_stats", "sol_attn_forward_host",
     "sol_attn_stage_pool", "sol_attn_stage_threshold", "sol_attn_stage_fused",
     "sol_attn_workspace_bytes", "sol_attn_release", "sol_attn_error_string",
-    "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc",
+    "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc", "sol_attn_profile_read",
 )
 
 
@@ -81,9 +83,10 @@ def lib():
     L.sol_attn_error_string.restype = ctypes.c_char_p
     L.sol_attn_kernels_per_forward.argtypes = []
     L.sol_attn_forward_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    L.sol_attn_profile_read.argtypes = [vp, i, i]
     for name in ("sol_attn_forward", "sol_attn_forward_ex", "sol_attn_stats", "sol_attn_forward_host",
                  "sol_attn_stage_pool", "sol_attn_stage_threshold", "sol_attn_stage_fused", "sol_attn_release",
-                 "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc"):
+                 "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc", "sol_attn_profile_read"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -215,6 +218,22 @@ def stage_fused(q, k, v, out, chunk: int, *, flags: int = 0, debug: Optional[Deb
 
 def workspace_bytes(B: int, H: int, L: int, d: int) -> int:
     return int(lib().sol_attn_workspace_bytes(B, H, L, d, BLOCK))
+
+
+PROFILE_SLOTS = (
+    "route.wait_item_empty", "k.wait_item", "k.wait_q_empty", "k.wait_stage", "v.wait_item", "v.wait_stage",
+    "mma.wait_p", "mma.wait_v", "mma.wait_item", "mma.wait_q", "mma.wait_s_empty", "mma.wait_k",
+    "softmax.wait_item", "softmax.wait_s", "softmax.wait_o", "softmax.wait_exchange",
+    "total.route", "total.k", "total.v", "total.mma", "total.softmax",
+    "softmax.pass1", "softmax.rescale", "softmax.pass2", "softmax.epilogue", "softmax.tiles", "softmax.rescales",
+)
+
+
+def profile_read(reset: bool = True) -> dict:
+    """Cycle counters of the profiling build, summed over CTAs (see sol_attn_profile_read)."""
+    buf = (ctypes.c_uint64 * 32)()
+    _check(lib().sol_attn_profile_read(buf, 32, 1 if reset else 0))
+    return {name: int(buf[k]) for k, name in enumerate(PROFILE_SLOTS)}
 
 
 def release():

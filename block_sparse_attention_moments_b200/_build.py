@@ -8,6 +8,7 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libsol_attn.so")
+PROFILE_LIB = os.path.join(PKG, "libsol_attn_profile.so")
 SOURCES = [os.path.join(PKG, "csrc", "sol_attn.cu")]
 DEPS = [os.path.join(PKG, "csrc", f) for f in ("fused.cuh", "moments.cuh", "pool.cuh", "sm100_ptx.cuh")] + [
     os.path.join(ROOT, "include", "sol_attn.h")]
@@ -26,17 +27,21 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found; the CUDA toolkit is required to build libsol_attn.so")
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB):
+def is_stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in SOURCES + DEPS)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and not is_stale():
-        return LIB
-    cmd = [nvcc_path(), *NVCC_FLAGS, *extra_flags, "-I", os.path.join(ROOT, "include"), "-o", LIB, *SOURCES]
+def build(force: bool = False, verbose: bool = False, extra_flags=(), profile: bool = False) -> str:
+    """Build libsol_attn.so (or, with profile=True, libsol_attn_profile.so with the
+    fused kernel's cycle accounting compiled in)."""
+    lib = PROFILE_LIB if profile else LIB
+    if not force and not is_stale(lib):
+        return lib
+    flags = [*NVCC_FLAGS, *extra_flags] + (["-DSOL_ATTN_PROFILE"] if profile else [])
+    cmd = [nvcc_path(), *flags, "-I", os.path.join(ROOT, "include"), "-o", lib, *SOURCES]
     if verbose:
         print(" ".join(cmd))
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -44,10 +49,10 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
     if verbose and (r.stdout or r.stderr):
         print(r.stdout, r.stderr)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
     import sys
-    print(build(force="--force" in sys.argv, verbose=True,
+    print(build(force="--force" in sys.argv, verbose=True, profile="--profile" in sys.argv,
                 extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []))

@@ -26,13 +26,14 @@
 //           O += P·[V_a;V_b].
 // Epilogue: O / l in bf16 for rows < L.
 //
-// Warp roles (256 threads, one persistent CTA per SM, atomic work counter):
-//   warps 0-3  softmax: one thread per tile row; masks, lazy-rescaled online
+// Warp roles (384 threads, one persistent CTA per SM, atomic work counter):
+//   warps 0-7  softmax, two warpgroups: each thread owns one tile row and one
+//              half of the tile's columns; masks, lazy-rescaled online
 //              softmax, P to shared memory, O correction in TMEM, epilogue.
-//   warp 4     producer of Q and of the K side (K blocks, or K̄ hi/lo) by TMA.
-//   warp 5     tcgen05 MMA issuer: S(t+1) is issued before PV(t).
-//   warp 6     producer of the V side (V blocks, or V̂) by TMA.
-//   warp 7     routing: fetches the next item, computes ŝ_ij = Q̄_i·K̄_j/sqrt(d)
+//   warp 8     producer of Q and of the K side (K blocks, or K̄ hi/lo) by TMA.
+//   warp 9     tcgen05 MMA issuer: S(t+1) is issued before PV(t).
+//   warp 10    producer of the V side (V blocks, or V̄) by TMA.
+//   warp 11    routing: fetches the next item, computes ŝ_ij = Q̄_i·K̄_j/sqrt(d)
 //              in fp32 for both halves, compares with τ_i (warp ballot -> mask
 //              words), one item ahead of the others (double-buffered slots).
 // Every role walks the same tile sequence, derived from the item's masks.
@@ -52,6 +53,23 @@
 namespace solattn {
 
 constexpr int kMaxMaskWords = 512;       // N <= 16384 pooled blocks per head
+
+// Optional per-role cycle accounting (build with -DSOL_ATTN_PROFILE): every
+// bounded wait and the softmax phases add their clock64() cycles to a slot;
+// the per-CTA totals are summed into g_profile at exit.
+enum ProfSlot : int {
+  kPrRouteWait, kPrKItem, kPrKQEmpty, kPrKEmpty, kPrVItem, kPrVEmpty,
+  kPrMmaP, kPrMmaV, kPrMmaItem, kPrMmaQ, kPrMmaSEmpty, kPrMmaK,
+  kPrSmItem, kPrSmS, kPrSmO, kPrSmX,
+  kPrTotRoute, kPrTotK, kPrTotV, kPrTotMma, kPrTotSm,
+  kPrSmPass1, kPrSmRescale, kPrSmPass2, kPrSmEpi, kPrSmTiles, kPrSmRescales, kPrSlots
+};
+#ifdef SOL_ATTN_PROFILE
+__device__ unsigned long long g_profile[32];
+#define SA_PROF(x) x
+#else
+#define SA_PROF(x)
+#endif
 constexpr unsigned kFlagSelectAll = 1u;
 constexpr unsigned kFlagExactOnly = 2u;
 constexpr unsigned kStatusTimeout = 1u;
@@ -92,6 +110,8 @@ struct __align__(16) FusedCtl {
   uint64_t v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, o_done;
+  uint64_t xchg;                    // softmax warpgroups: partial row max / sum exchange
+  float xval[2][2][128];            // [phase parity][warpgroup][row]
   uint32_t tmem_base;
   int abort;
 };
@@ -107,8 +127,8 @@ constexpr uint32_t kSmemCtl = kSmemP + kTile;
 constexpr uint32_t kFusedSmemBytes = kSmemCtl + sizeof(FusedCtl) + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0, kTmemS0 = 128;
-constexpr int kThreads = 256;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxThreads = 256;   // two warpgroups, each owning half of a tile's columns
 constexpr uint32_t kItemEmptyCount = kSoftmaxThreads + 3;  // softmax rows + K producer + V producer + MMA
 
 __device__ __forceinline__ bool mask_bit(const uint32_t* m, int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
@@ -228,8 +248,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
                           const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_vb,
                           const FusedParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base for the swizzled tiles.  Offsetting the shared array
+  // itself (not a round trip through an integer) keeps every pointer below in
+  // the shared state space, so accesses compile to shared-memory instructions.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem + kSmemQ;
   uint8_t* sK = smem + kSmemK;
   uint8_t* sV = smem + kSmemV;
@@ -259,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ctl.q_empty, 1);
     mbar_init(&ctl.p_full, kSoftmaxThreads);
     mbar_init(&ctl.o_done, 1);
+    mbar_init(&ctl.xchg, kSoftmaxThreads);
     ctl.abort = 0;
     fence_mbar_init();
   }
@@ -274,18 +298,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Bounded wait; on a timeout raise the abort flag and the status word.  All
   // later waits return false at once, every role leaves its loop, and the CTA
   // meets at the final barrier.
-  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-    if (mbar_wait(bar, parity, abort_flag, p.timeout_ns)) return true;
+  SA_PROF(unsigned long long prof[kPrSlots]; for (int i = 0; i < kPrSlots; ++i) prof[i] = 0;
+          const unsigned long long prof_t0 = clock64();)
+  auto wait = [&](uint64_t* bar, uint32_t parity, int slot) -> bool {
+    SA_PROF(const unsigned long long tw = clock64();)
+    const bool okw = mbar_wait(bar, parity, abort_flag, p.timeout_ns);
+    SA_PROF(prof[slot] += clock64() - tw;)
+    (void)slot;
+    if (okw) return true;
     *abort_flag = 1;
     atomicOr(p.status, kStatusTimeout);
     return false;
   };
 
-  if (warp == 7) {
+  if (warp == 11) {
     // =========================================================== routing
     for (int seq = 0;; ++seq) {
       const int s = seq & 1;
-      if (seq >= 2 && !wait(&ctl.item_empty[s], ((seq >> 1) - 1) & 1)) break;
+      if (seq >= 2 && !wait(&ctl.item_empty[s], ((seq >> 1) - 1) & 1, kPrRouteWait)) break;
       int item = 0;
       if (lane == 0) item = static_cast<int>(atomicAdd(p.work_counter, 1u));
       item = __shfl_sync(0xFFFFFFFFu, item, 0);
@@ -357,15 +387,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.item_full[s]);   // release: masks and item visible
     }
-  } else if (warp == 4 || warp == 6) {
+  } else if (warp == 8 || warp == 10) {
     // =========================================================== TMA producers
-    const bool kside = (warp == 4);
+    const bool kside = (warp == 8);
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       for (int seq = 0;; ++seq) {
         const int s = seq & 1;
-        if (!wait(&ctl.item_full[s], (seq >> 1) & 1)) break;
+        if (!wait(&ctl.item_full[s], (seq >> 1) & 1, kside ? kPrKItem : kPrVItem)) break;
         const ItemSlot& sl = ctl.slot[s];
         const int item = sl.item;
         if (item < 0) break;
@@ -373,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pair = item - bh * p.num_pairs;
         bool ok = true;
         if (kside) {  // query tile of the item (the previous item's S MMAs must be done)
-          if (seq > 0 && !wait(&ctl.q_empty, (seq - 1) & 1)) break;
+          if (seq > 0 && !wait(&ctl.q_empty, (seq - 1) & 1, kPrKQEmpty)) break;
           mbar_arrive_expect_tx(&ctl.q_full, 128u * D * 2u);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
@@ -385,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (it.next(t)) {
           uint64_t* empty = kside ? &ctl.k_empty[stage] : &ctl.v_empty[stage];
           uint64_t* full = kside ? &ctl.k_full[stage] : &ctl.v_full[stage];
-          if (!wait(empty, phase ^ 1u)) { ok = false; break; }
+          if (!wait(empty, phase ^ 1u, kside ? kPrKEmpty : kPrVEmpty)) { ok = false; break; }
           uint8_t* dst = (kside ? sK : sV) + stage * kTile;
           if (t.kind == 0) {
             mbar_arrive_expect_tx(full, (kside ? 2u : 1u) * p.W * D * 2u);
@@ -417,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // =========================================================== MMA issuer
     if (lane == 0) {
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
@@ -433,8 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       // O (+)= P · Vside for the pending tile.
       auto issue_pv = [&]() -> bool {
-        if (!wait(&ctl.p_full, pv_idx & 1)) return false;
-        if (!wait(&ctl.v_full[pv_stage], pv_phase)) return false;
+        if (!wait(&ctl.p_full, pv_idx & 1, kPrMmaP)) return false;
+        if (!wait(&ctl.v_full[pv_stage], pv_phase, kPrMmaV)) return false;
         tc_fence_after();
         const int ksteps = pt.ncols / 16;
         const uint32_t vbase = sVa + pv_stage * kTile;
@@ -450,20 +480,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int seq = 0;; ++seq) {
         const int s = seq & 1;
-        if (!wait(&ctl.item_full[s], (seq >> 1) & 1)) { ok = false; break; }
+        if (!wait(&ctl.item_full[s], (seq >> 1) & 1, kPrMmaItem)) { ok = false; break; }
         const ItemSlot& sl = ctl.slot[s];
         const int item = sl.item;
         if (item < 0) break;
         const int pair = item % p.num_pairs;
-        if (!wait(&ctl.q_full, seq & 1)) { ok = false; break; }
+        if (!wait(&ctl.q_full, seq & 1, kPrMmaQ)) { ok = false; break; }
         TileIter it;
         it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
         Tile t;
         while (it.next(t)) {
           // S(t) = Q · Kside^T into S buffer (tcount & 1)
           const int b = tcount & 1;
-          if (tcount >= 2 && !wait(&ctl.s_empty[b], ((tcount >> 1) - 1) & 1)) { ok = false; break; }
-          if (!wait(&ctl.k_full[kstage], kphase)) { ok = false; break; }
+          if (tcount >= 2 && !wait(&ctl.s_empty[b], ((tcount >> 1) - 1) & 1, kPrMmaSEmpty)) { ok = false; break; }
+          if (!wait(&ctl.k_full[kstage], kphase, kPrMmaK)) { ok = false; break; }
           tc_fence_after();
           const uint32_t dS = tmem + kTmemS0 + b * 128;
           const uint32_t kbase = sKa + kstage * kTile;
@@ -509,18 +539,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && pend) issue_pv();
     }
   } else {
-    // =========================================================== softmax (warps 0-3)
-    const int row = tid;              // tile row = TMEM lane
+    // =========================================================== softmax (warps 0-7)
+    // Two warpgroups share every tile row: warpgroup wg owns half of the
+    // tile's 32-column groups (and half of O's columns).  Partial row maxima
+    // and, at the end of an item, partial row sums are exchanged through
+    // shared memory behind a bounded mbarrier.
+    const int wg = warp >> 2;
+    const int row = tid & 127;        // tile row = TMEM lane
     const int half = row >> 6;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + kTmemO + lane_base;
     const int tail_n = p.L - 64 * (p.N - 1);
+    constexpr int OG = D / 64;        // 32-column groups of O per warpgroup
     uint32_t tcount = 0;     // tiles processed
     uint32_t pv_seen = 0;    // PV completions waited for
-    bool ok = true;
-    for (int seq = 0; ok; ++seq) {
+    uint32_t xc = 0;         // exchanges done
+    // Exchange one value per row with the other warpgroup; returns the other's.
+    auto exchange = [&](float v) -> float {
+      const int ph = xc & 1;
+      ctl.xval[ph][wg][row] = v;
+      mbar_arrive(&ctl.xchg);
+      wait(&ctl.xchg, ph, kPrSmX);
+      ++xc;
+      return ctl.xval[ph][wg ^ 1][row];
+    };
+    for (int seq = 0;; ++seq) {
       const int s = seq & 1;
-      if (!wait(&ctl.item_full[s], (seq >> 1) & 1)) break;
+      if (!wait(&ctl.item_full[s], (seq >> 1) & 1, kPrSmItem)) break;
       const ItemSlot& sl = ctl.slot[s];
       const int item = sl.item;
       if (item < 0) break;
@@ -533,16 +578,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileIter it;
       it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
       Tile t;
+      // After a timeout every wait returns at once; the loop still runs its
+      // (bounded) course so both warpgroups keep making the same calls.
       while (it.next(t)) {
         any_tile = true;
         const int b = tcount & 1;
-        if (!wait(&ctl.s_full[b], (tcount >> 1) & 1)) { ok = false; break; }
+        wait(&ctl.s_full[b], (tcount >> 1) & 1, kPrSmS);
         tc_fence_after();
         const uint32_t tS = tmem + kTmemS0 + b * 128 + lane_base;
-        // Two passes over the tile in 32-column groups, each reading S from
-        // TMEM: the first finds the row maximum, the second writes P.  Keeping
-        // one group in registers at a time keeps the loop body small.
+        // this warpgroup's 32-column groups of the tile
         const int ng = t.ncols >> 5;
+        const int gper = (ng >= 2) ? (ng >> 1) : 1;
+        const int g0 = (ng >= 2) ? wg * gper : wg;
+        const int g1 = min(g0 + gper, ng);
         // validity of a group's 32 columns (warp-uniform: a warp's rows share a half)
         auto group_bits = [&](int g) -> uint32_t {
           const int c0 = 32 * g;
@@ -557,34 +605,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
           return mask_bit(own, jx) ? range : 0u;
         };
+        SA_PROF(unsigned long long tph = clock64(); prof[kPrSmTiles] += 1;)
+        // Pass 1 reads this thread's 32-column groups from TMEM for the row
+        // maximum; pass 2 reads them again for the probabilities.  Both passes
+        // are runtime loops over one copy of the group code, which keeps the
+        // softmax loop small enough to stay in the instruction cache.
+        // Column adjustments of a group, applied only when needed: invalid
+        // columns become -inf, and the ragged last block's approximation
+        // column gets log2(tail_n / 64) added (its weight is tail_n, not 64).
+        const int tail_col = (t.kind == 0 && tail_n != 64) ? (p.N - 1 - t.ja) : -1;
+        const int tail_g = (tail_col >= 0 && tail_col < t.ncols) ? (tail_col >> 5) : -1;
+        const float tail_raw = (log2f(static_cast<float>(tail_n)) - 6.f) / p.scale_log2;
+        auto adjust = [&](float (&xv)[32], int g) {
+          const uint32_t bits = group_bits(g);
+          const int et = (g == tail_g) ? (tail_col & 31) : -1;
+          if (bits != 0xFFFFFFFFu || et >= 0) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (e == et) xv[e] += tail_raw;
+              if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
+            }
+          }
+        };
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll 1
-        for (int g = 0; g < ng; ++g) {
+        for (int g = g0; g < g1; ++g) {
           float xv[32];
           tmem_ld_x32f(tS + 32 * g, xv);
           tmem_ld_wait();
           reg_fence32(xv);
-          const uint32_t bits = group_bits(g);
-          if (bits != 0xFFFFFFFFu) {
+          adjust(xv, g);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
-          }
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            mx0 = fmaxf(mx0, xv[e]);
-            mx1 = fmaxf(mx1, xv[e + 1]);
-            mx2 = fmaxf(mx2, xv[e + 2]);
-            mx3 = fmaxf(mx3, xv[e + 3]);
+          for (int e = 0; e < 32; e += 8) {
+            mx0 = max3f(mx0, xv[e], xv[e + 1]);
+            mx1 = max3f(mx1, xv[e + 2], xv[e + 3]);
+            mx2 = max3f(mx2, xv[e + 4], xv[e + 5]);
+            mx3 = max3f(mx3, xv[e + 6], xv[e + 7]);
           }
         }
-        const float rmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float pmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        SA_PROF(prof[kPrSmPass1] += clock64() - tph;)
+        const float rmax = fmaxf(pmax, exchange(pmax));
         // In log2 units.  An approximation column stands for its n_j tokens:
         // its weight n_j is folded into the logit as + log2(n_j) (6 for a full
         // block) and the value side uses the block mean V̂_j / n_j.
         const float boost = (t.kind == 0) ? 6.f : 0.f;
         const float tmax = (rmax == -INFINITY) ? -INFINITY : fmaf(rmax, p.scale_log2, boost);
-        // lazy rescale: move the reference max only when it grows by > 8 (x256)
+        // lazy rescale: move the reference max only when it grows by > 8 (x256);
+        // both warpgroups take the same decision from the same row maximum
         const bool need = tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY);
         float alpha = 1.f;
         if (need) {
@@ -594,19 +662,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_run = m_new;
         }
         const float off = boost - ((m_run == -INFINITY) ? 0.f : m_run);
-        // the ragged last block, when it is an approximation column, weighs tail_n
-        const int tail_col = (t.kind == 0 && tail_n != 64) ? (p.N - 1 - t.ja) : -1;
-        const int tail_g = (tail_col >= 0 && tail_col < t.ncols) ? (tail_col >> 5) : -1;
-        const float off_tail = off + (log2f(static_cast<float>(tail_n)) - 6.f);
         // the previous tile's PV must be done before P is overwritten or O rescaled
         if (pv_seen < tcount) {
-          if (!wait(&ctl.o_done, (tcount - 1) & 1)) { ok = false; break; }
+          wait(&ctl.o_done, (tcount - 1) & 1, kPrSmO);
           pv_seen = tcount;
           tc_fence_after();
         }
+        SA_PROF(tph = clock64();)
         if (!t.first && __any_sync(0xFFFFFFFFu, need)) {
+          SA_PROF(prof[kPrSmRescales] += 1;)
 #pragma unroll 1
-          for (int c32 = 0; c32 < D / 32; ++c32) {
+          for (int c32 = wg * OG; c32 < (wg + 1) * OG; ++c32) {
             uint32_t r[32];
             tmem_ld_x32(tO + c32 * 32, r);
             tmem_ld_wait();
@@ -616,48 +682,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st_wait();
         }
-        float sm0 = 0.f, sm1 = 0.f, sm2 = 0.f, sm3 = 0.f;
+        SA_PROF(prof[kPrSmRescale] += clock64() - tph; tph = clock64();)
+        // pass 2: probabilities, partial row sum, P to shared memory.  12 of
+        // every 32 exponentials run on the FMA/ALU pipes (exp2_poly), the rest
+        // on MUFU; masked columns hold -inf and give 0 either way.
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 of2 = make_float2(off, off);
+        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
 #pragma unroll 1
-        for (int g = 0; g < ng; ++g) {
+        for (int g = g0; g < g1; ++g) {
           float xv[32];
           tmem_ld_x32f(tS + 32 * g, xv);
           tmem_ld_wait();
           reg_fence32(xv);
-          const uint32_t bits = group_bits(g);
-          if (bits != 0xFFFFFFFFu) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
-          }
+          adjust(xv, g);
           uint32_t pk[16];
-          if (g != tail_g) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float p0 = ex2_approx(fmaf(xv[e], p.scale_log2, off));
-              const float p1 = ex2_approx(fmaf(xv[e + 1], p.scale_log2, off));
-              const float p2 = ex2_approx(fmaf(xv[e + 2], p.scale_log2, off));
-              const float p3 = ex2_approx(fmaf(xv[e + 3], p.scale_log2, off));
-              sm0 += p0;
-              sm1 += p1;
-              sm2 += p2;
-              sm3 += p3;
-              pk[e >> 1] = pack_bf16x2(p0, p1);
-              pk[(e >> 1) + 1] = pack_bf16x2(p2, p3);
-            }
-          } else {
-            const int et = tail_col & 31;
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float p0 = ex2_approx(fmaf(xv[e], p.scale_log2, e == et ? off_tail : off));
-              const float p1 = ex2_approx(fmaf(xv[e + 1], p.scale_log2, e + 1 == et ? off_tail : off));
-              sm0 += p0;
-              sm1 += p1;
-              pk[e >> 1] = pack_bf16x2(p0, p1);
-            }
+          for (int e = 0; e < 32; e += 8) {
+            const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
+            const float2 y1 = __ffma2_rn(make_float2(xv[e + 2], xv[e + 3]), sc2, of2);
+            const float2 y2 = __ffma2_rn(make_float2(xv[e + 4], xv[e + 5]), sc2, of2);
+            const float2 y3 = __ffma2_rn(make_float2(xv[e + 6], xv[e + 7]), sc2, of2);
+            const float2 q0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+            const float2 q1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+            const float2 q2 = make_float2(ex2_approx(y2.x), exp2_poly(y2.y));
+            const float2 q3 = make_float2(exp2_poly(y3.x), exp2_poly(y3.y));
+            sa = __fadd2_rn(sa, __fadd2_rn(q0, q2));
+            sb = __fadd2_rn(sb, __fadd2_rn(q1, q3));
+            pk[e >> 1] = pack_bf16x2(q0.x, q0.y);
+            pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
+            pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
+            pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
           }
           store_p32(sP, row, 32 * g, pk);
         }
-        l_run += (sm0 + sm1) + (sm2 + sm3);
+        l_run += (sa.x + sa.y) + (sb.x + sb.y);
+        SA_PROF(prof[kPrSmPass2] += clock64() - tph;)
         // S buffer b may now be overwritten by the MMA of tile tcount + 2
         tc_fence_before();
         mbar_arrive(&ctl.s_empty[b]);
@@ -666,18 +726,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&ctl.p_full);
         ++tcount;
       }
-      if (!ok) break;
-      // ---- epilogue: wait for the item's last PV, O / l for rows < L (Eq. 10)
+      // ---- epilogue: row sum of both warpgroups, last PV, O / l for rows < L (Eq. 10)
+      SA_PROF(const unsigned long long tep = clock64();)
+      const float l_tot = l_run + exchange(l_run);
       if (tcount > pv_seen) {
-        if (!wait(&ctl.o_done, (tcount - 1) & 1)) break;
+        wait(&ctl.o_done, (tcount - 1) & 1, kPrSmO);
         pv_seen = tcount;
         tc_fence_after();
       }
       const int token = 128 * pair + row;
-      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
       uint16_t* orow = p.out + (static_cast<size_t>(bh) * p.L + token) * D;
-#pragma unroll
-      for (int c32 = 0; c32 < D / 32; ++c32) {
+#pragma unroll 1
+      for (int c32 = wg * OG; c32 < (wg + 1) * OG; ++c32) {
         uint32_t r[32];
         if (any_tile) {            // an item with no tile (exact-only, nothing selected) outputs 0
           tmem_ld_x32(tO + c32 * 32, r);
@@ -698,11 +759,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      SA_PROF(prof[kPrSmEpi] += clock64() - tep;)
       tc_fence_before();
       mbar_arrive(&ctl.item_empty[s]);
     }
   }
 
+  SA_PROF({
+    const int tslot = warp == 11 ? kPrTotRoute : warp == 8 ? kPrTotK : warp == 10 ? kPrTotV
+                    : warp == 9 ? kPrTotMma : kPrTotSm;
+    if (lane == 0 && (warp >= 8 || warp == 0)) {
+      prof[tslot] = clock64() - prof_t0;
+      for (int i = 0; i < kPrSlots; ++i) if (prof[i]) atomicAdd(&g_profile[i], prof[i]);
+    }
+  })
   // After a timeout, give copies or MMAs that may still be in flight a bounded
   // time to land before the shared memory and TMEM are released.
   __syncwarp();

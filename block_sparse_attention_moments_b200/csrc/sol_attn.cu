@@ -560,6 +560,24 @@ const char* sol_attn_error_string(int code) {
 
 int sol_attn_kernels_per_forward(void) { return 4; }
 
+int sol_attn_profile_read(uint64_t* cycles, int n, int reset) {
+#ifdef SOL_ATTN_PROFILE
+  if (!cycles || n < 1) return fail(SOL_ATTN_ERR_ARG, "cycles is NULL or n < 1");
+  unsigned long long h[32];
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpyFromSymbol(h, g_profile, sizeof(h)));
+  for (int i = 0; i < n && i < 32; ++i) cycles[i] = h[i];
+  if (reset) {
+    unsigned long long z[32] = {0};
+    CUDA_TRY(cudaMemcpyToSymbol(g_profile, z, sizeof(z)));
+  }
+  return SOL_ATTN_OK;
+#else
+  (void)cycles; (void)n; (void)reset;
+  return fail(SOL_ATTN_ERR_UNSUPPORTED, "library built without SOL_ATTN_PROFILE");
+#endif
+}
+
 int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B, int H, int L, int d,
                              int block, int chunk, float beta, void* stream) {
   int rc;
