@@ -233,7 +233,8 @@ def run_role_profile(args):
         print(json.dumps({"workload": wl.name, "mode": tag, "ctas": nsm, "tiles_per_cta": tiles / nsm,
                           "cycles_per_cta": {k2: round(v2) for k2, v2 in per_cta.items()},
                           "softmax_cycles_per_tile": {k2: round(prof[k2] / tiles, 1) for k2 in
-                                                      ("softmax.pass1", "softmax.rescale", "softmax.pass2",
+                                                      ("softmax.wait_desc", "softmax.pass1",
+                                                       "softmax.rescale", "softmax.pass2", "softmax.epilogue",
                                                        "softmax.wait_s", "softmax.wait_o",
                                                        "softmax.wait_exchange")}}), flush=True)
 

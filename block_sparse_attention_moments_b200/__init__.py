@@ -221,11 +221,12 @@ def workspace_bytes(B: int, H: int, L: int, d: int) -> int:
 
 
 PROFILE_SLOTS = (
-    "route.wait_item_empty", "k.wait_item", "k.wait_q_empty", "k.wait_stage", "v.wait_item", "v.wait_stage",
-    "mma.wait_p", "mma.wait_v", "mma.wait_item", "mma.wait_q", "mma.wait_s_empty", "mma.wait_k",
-    "softmax.wait_item", "softmax.wait_s", "softmax.wait_o", "softmax.wait_exchange",
+    "route.wait_item_empty", "k.wait_desc", "k.wait_q_empty", "k.wait_stage", "v.wait_desc", "v.wait_stage",
+    "mma.wait_p", "mma.wait_v", "mma.wait_desc", "mma.wait_q", "mma.wait_s_empty", "mma.wait_k",
+    "softmax.wait_desc", "softmax.wait_s", "softmax.wait_o", "softmax.wait_exchange",
     "total.route", "total.k", "total.v", "total.mma", "total.softmax",
     "softmax.pass1", "softmax.rescale", "softmax.pass2", "softmax.epilogue", "softmax.tiles", "softmax.rescales",
+    "sched.wait_item", "sched.wait_ring", "total.sched",
 )
 
 

@@ -30,17 +30,28 @@
 //   warps 0-7  softmax, two warpgroups: each thread owns one tile row and one
 //              half of the tile's columns; masks, lazy-rescaled online
 //              softmax, P to shared memory, O correction in TMEM, epilogue.
-//   warp 8     producer of Q and of the K side (K blocks, or K̄ hi/lo) by TMA.
+//   warp 8     TMA producers: lane 0 loads Q and the K side (K blocks, or K̄
+//              hi/lo), lane 1 the V side (V blocks, or V̄).
 //   warp 9     tcgen05 MMA issuer: S(t+1) is issued before PV(t).
-//   warp 10    producer of the V side (V blocks, or V̄) by TMA.
-//   warp 11    routing: fetches the next item, computes ŝ_ij = Q̄_i·K̄_j/sqrt(d)
+//   warp 10    routing: fetches the next item, computes ŝ_ij = Q̄_i·K̄_j/sqrt(d)
 //              in fp32 for both halves, compares with τ_i (warp ballot -> mask
-//              words), one item ahead of the others (double-buffered slots).
-// Every role walks the same tile sequence, derived from the item's masks.
+//              words), one item ahead (double-buffered mask slots).
+//   warp 11    scheduler: walks each item's tile sequence from its masks and
+//              publishes one descriptor per tile (blocks, column validity per
+//              half, first/last flags) into a shared-memory ring that the
+//              producers, the MMA issuer and the softmax warps consume.
+//
+// Tiles alternate between the two softmax warpgroups (global tile index
+// parity w): warpgroup w owns every row of its tiles, keeps its own running
+// max / sum, and accumulates into its own O_w.  At the end of an item the two
+// partial results are merged, O = (2^(m0-m) O_0 + 2^(m1-m) O_1) / (2^(m0-m) l_0
+// + 2^(m1-m) l_1), the usual combination of partial online softmaxes.  P is
+// written back into TMEM over its S tile (bf16 pairs) and fed to the PV MMA
+// as its A operand, so the only shared-memory operand traffic is Q, K and V.
 //
 // Shared memory (1024-byte aligned, 128-byte swizzled tiles):
-//   Q 32 KB | K ring 2 x 32 KB | V ring 2 x 32 KB | P 32 KB | control.
-// TMEM (512 columns): O [0,128), S buffers [128,256) and [256,384).
+//   Q 32 KB | K ring 2 x 32 KB | V ring 2 x 32 KB | control.
+// TMEM (512 columns): O_0 [0,128), O_1 [128,256), S_0/P_0 [256,384), S_1/P_1 [384,512).
 #pragma once
 
 #include <cstddef>
@@ -58,11 +69,12 @@ constexpr int kMaxMaskWords = 512;       // N <= 16384 pooled blocks per head
 // bounded wait and the softmax phases add their clock64() cycles to a slot;
 // the per-CTA totals are summed into g_profile at exit.
 enum ProfSlot : int {
-  kPrRouteWait, kPrKItem, kPrKQEmpty, kPrKEmpty, kPrVItem, kPrVEmpty,
-  kPrMmaP, kPrMmaV, kPrMmaItem, kPrMmaQ, kPrMmaSEmpty, kPrMmaK,
-  kPrSmItem, kPrSmS, kPrSmO, kPrSmX,
+  kPrRouteWait, kPrKDesc, kPrKQEmpty, kPrKEmpty, kPrVDesc, kPrVEmpty,
+  kPrMmaP, kPrMmaV, kPrMmaDesc, kPrMmaQ, kPrMmaSEmpty, kPrMmaK,
+  kPrSmDesc, kPrSmS, kPrSmO, kPrSmX,
   kPrTotRoute, kPrTotK, kPrTotV, kPrTotMma, kPrTotSm,
-  kPrSmPass1, kPrSmRescale, kPrSmPass2, kPrSmEpi, kPrSmTiles, kPrSmRescales, kPrSlots
+  kPrSmPass1, kPrSmRescale, kPrSmPass2, kPrSmEpi, kPrSmTiles, kPrSmRescales, kPrSchedItem, kPrSchedRing,
+  kPrTotSched, kPrSlots
 };
 #ifdef SOL_ATTN_PROFILE
 __device__ unsigned long long g_profile[32];
@@ -82,6 +94,7 @@ struct FusedParams {
   unsigned flags;
   float scale_log2;         // log2(e) / sqrt(d)
   float inv_sqrt_d;
+  float tail_raw;           // (log2(n_tail) - 6) / scale_log2: logit shift of the ragged block's approximation
   const float* qbar;        // [BH][N][d] fp32
   const float* kbar;        // [BH][N][d] fp32
   const float* tau;         // [BH][N] fp32
@@ -95,23 +108,42 @@ struct FusedParams {
 
 constexpr int kStages = 2;
 
+// One entry of the tile sequence, published by the scheduler warp.
+struct __align__(16) TileDesc {
+  uint32_t bits[2][4];  // [half][32-column group]: columns that take part for that half's rows
+  int ja, jb;           // approximation: first pooled key; exact: key blocks (jb = -1: one block)
+  int bh, pair;         // work item
+  int ncols;            // 32, 64 or 128 (MMA N of S, K of PV)
+  int flags;            // kDesc* bits
+  int tail;             // column of the ragged block's approximation (weight n_tail), or -1
+  int pad;
+};
+constexpr int kDescFirst = 1;    // first tile of its item (PV overwrites O)
+constexpr int kDescLast = 2;     // last tile of its item
+constexpr int kDescApprox = 4;   // approximation tile (else exact)
+constexpr int kDescEmpty = 8;    // item without any tile (exact-only, nothing selected)
+constexpr int kDescEnd = 16;     // no more work
+constexpr int kRing = 8;         // descriptor ring entries
+
 struct __align__(16) ItemSlot {
   uint32_t mask[2][kMaxMaskWords];  // selection bits of both halves
   int item;                         // work item index, or -1 = no more work
-  int pad[3];
+  int no_tiles;                     // exact-only item with nothing selected: no tile at all
+  int pad[2];
 };
 
 struct __align__(16) FusedCtl {
   ItemSlot slot[2];
+  TileDesc ring[kRing];             // scheduler -> producers, MMA issuer, softmax
   float qbar[2][128];               // routing: pooled queries of the pair
   uint64_t item_full[2], item_empty[2];
+  uint64_t ring_full[kRing], ring_empty[kRing];
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full, o_done;
+  uint64_t s_full[2], p_full[2], o_done[2];   // per softmax warpgroup (tile parity)
   uint64_t xchg;                    // softmax warpgroups: partial row max / sum exchange
-  float xval[2][2][128];            // [phase parity][warpgroup][row]
+  float xval[2][2][2][128];         // [phase parity][warpgroup][value][row]
   uint32_t tmem_base;
   int abort;
 };
@@ -122,14 +154,13 @@ constexpr uint32_t kTile = 32768;  // 128 rows x 128 bf16
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + kTile;
 constexpr uint32_t kSmemV = kSmemK + kStages * kTile;
-constexpr uint32_t kSmemP = kSmemV + kStages * kTile;
-constexpr uint32_t kSmemCtl = kSmemP + kTile;
+constexpr uint32_t kSmemCtl = kSmemV + kStages * kTile;
 constexpr uint32_t kFusedSmemBytes = kSmemCtl + sizeof(FusedCtl) + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0, kTmemS0 = 128;
+constexpr uint32_t kTmemO0 = 0, kTmemS0 = 256;   // O_w at 128 w, S_w / P_w at 256 + 128 w
 constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;   // two warpgroups, each owning half of a tile's columns
-constexpr uint32_t kItemEmptyCount = kSoftmaxThreads + 3;  // softmax rows + K producer + V producer + MMA
+constexpr uint32_t kRingEmptyCount = 8 + 3;  // softmax warps (lane 0 each) + K producer + V producer + MMA
 
 __device__ __forceinline__ bool mask_bit(const uint32_t* m, int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
 
@@ -151,7 +182,7 @@ struct Tile {
 
 // Walks an item's tile sequence: for each chunk, approximation sub-tiles
 // (skipped when both halves selected every block in them), then the union of
-// the selected blocks, two per tile.  Every warp role runs its own copy.
+// the selected blocks, two per tile.  Run by the scheduler warp.
 struct TileIter {
   const uint32_t* m0;
   const uint32_t* m1;
@@ -229,18 +260,6 @@ struct TileIter {
   }
 };
 
-// Write one row's 32 probabilities (columns [c0, c0+32)), already packed as
-// bf16 pairs, into the 128B-swizzled K-major P tile.
-__device__ __forceinline__ void store_p32(uint8_t* sP, int row, int c0, const uint32_t* pk) {
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {  // four 16-byte chunks of 8 columns
-    const int c = c0 + 8 * g;
-    const int cb = c >> 6;                      // 64-column block
-    const int chunk = (c & 63) >> 3;            // 16-byte chunk within the 128-byte row
-    const uint32_t off = cb * 16384u + row * 128u + (((chunk ^ (row & 7)) & 7) << 4);
-    *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
-  }
-}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -256,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + kSmemQ;
   uint8_t* sK = smem + kSmemK;
   uint8_t* sV = smem + kSmemV;
-  uint8_t* sP = smem + kSmemP;
   FusedCtl& ctl = *reinterpret_cast<FusedCtl*>(smem + kSmemCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -268,9 +286,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl.item_full[s], 1);
-      mbar_init(&ctl.item_empty[s], kItemEmptyCount);
+      mbar_init(&ctl.item_empty[s], 1);
       mbar_init(&ctl.s_full[s], 1);
-      mbar_init(&ctl.s_empty[s], kSoftmaxThreads);
+      mbar_init(&ctl.p_full[s], kSoftmaxThreads / 2);
+      mbar_init(&ctl.o_done[s], 1);
+    }
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(&ctl.ring_full[r], 1);
+      mbar_init(&ctl.ring_empty[r], kRingEmptyCount);
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ctl.k_full[s], 1);
@@ -280,8 +303,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ctl.q_full, 1);
     mbar_init(&ctl.q_empty, 1);
-    mbar_init(&ctl.p_full, kSoftmaxThreads);
-    mbar_init(&ctl.o_done, 1);
     mbar_init(&ctl.xchg, kSoftmaxThreads);
     ctl.abort = 0;
     fence_mbar_init();
@@ -310,8 +331,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     atomicOr(p.status, kStatusTimeout);
     return false;
   };
+  // Consumer side of the descriptor ring: descriptor r lives in slot r % kRing.
+  auto ring_get = [&](uint32_t r, int slot) -> bool {
+    return wait(&ctl.ring_full[r % kRing], (r / kRing) & 1, slot);
+  };
 
-  if (warp == 11) {
+  if (warp == 10) {
     // =========================================================== routing
     for (int seq = 0;; ++seq) {
       const int s = seq & 1;
@@ -375,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.counts[static_cast<size_t>(bh) * p.N + i0] = cnt0;
         if (has1) p.counts[static_cast<size_t>(bh) * p.N + i1] = cnt1;
         sl.item = item;
+        sl.no_tiles = exact_only && (cnt0 + cnt1 == 0);
       }
       __syncwarp();
       if (p.mask_out) {
@@ -387,388 +413,456 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.item_full[s]);   // release: masks and item visible
     }
-  } else if (warp == 8 || warp == 10) {
+  } else if (warp == 11) {
+    // =========================================================== scheduler
+    uint32_t r = 0;   // descriptors published
+    const int NW = (p.N + 31) >> 5;
+    // Claim ring slot r (all consumers are done with descriptor r - kRing).
+    auto claim = [&]() -> TileDesc* {
+      if (r >= kRing && !wait(&ctl.ring_empty[r % kRing], ((r / kRing) - 1) & 1, kPrSchedRing)) return nullptr;
+      return &ctl.ring[r % kRing];
+    };
+    auto publish = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.ring_full[r % kRing]);   // release: descriptor visible
+      ++r;
+    };
+    for (int seq = 0;; ++seq) {
+      const int s = seq & 1;
+      if (!wait(&ctl.item_full[s], (seq >> 1) & 1, kPrSchedItem)) break;
+      const ItemSlot& sl = ctl.slot[s];
+      const int item = sl.item;
+      TileDesc* dsc = claim();
+      if (!dsc) break;
+      if (item < 0) {
+        if (lane == 0) dsc->flags = kDescEnd;
+        publish();
+        break;
+      }
+      const int bh = item / p.num_pairs;
+      const int pair = item - bh * p.num_pairs;
+      if (sl.no_tiles) {
+        if (lane == 0) {
+          dsc->bh = bh;
+          dsc->pair = pair;
+          dsc->flags = kDescEmpty;
+        }
+        publish();
+      } else {
+        TileIter it;
+        it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
+        Tile t, tn;
+        bool have = it.next(t);
+        bool first_desc = true;
+        while (have) {
+          const bool have_next = it.next(tn);
+          if (!first_desc && !(dsc = claim())) break;
+          first_desc = false;
+          // lanes 0-7 each compute one (half, 32-column group) validity word
+          if (lane < 8) {
+            const int g = lane >> 1, h = lane & 1;
+            uint32_t bits = 0u;
+            if (32 * g < t.ncols) {
+              if (t.kind == 0) {
+                const int nv = min(max(t.avalid - 32 * g, 0), 32);
+                const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+                bits = range & ~mask_bits32(sl.mask[h], t.ja + 32 * g, NW);
+              } else {
+                const int jx = (g < 2) ? t.ja : t.jb;
+                const int nv = min(max(p.L - (64 * jx + 32 * (g & 1)), 0), 32);
+                const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+                bits = mask_bit(sl.mask[h], jx) ? range : 0u;
+              }
+            }
+            dsc->bits[h][g] = bits;
+          } else if (lane == 8) {
+            const int tail_col = (t.kind == 0 && p.L - 64 * (p.N - 1) != 64) ? (p.N - 1 - t.ja) : -1;
+            dsc->ja = t.ja;
+            dsc->jb = t.jb;
+            dsc->bh = bh;
+            dsc->pair = pair;
+            dsc->ncols = t.ncols;
+            dsc->flags = (t.first ? kDescFirst : 0) | (have_next ? 0 : kDescLast) | (t.kind == 0 ? kDescApprox : 0);
+            dsc->tail = (tail_col >= 0 && tail_col < t.ncols) ? tail_col : -1;
+          }
+          publish();
+          t = tn;
+          have = have_next;
+        }
+        if (have) break;   // left early on a timeout
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.item_empty[s]);   // the item's masks are no longer read
+    }
+  } else if (warp == 8) {
     // =========================================================== TMA producers
-    const bool kside = (warp == 8);
-    if (lane == 0) {
+    const bool kside = (lane == 0);
+    if (lane < 2) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int seq = 0;; ++seq) {
-        const int s = seq & 1;
-        if (!wait(&ctl.item_full[s], (seq >> 1) & 1, kside ? kPrKItem : kPrVItem)) break;
-        const ItemSlot& sl = ctl.slot[s];
-        const int item = sl.item;
-        if (item < 0) break;
-        const int bh = item / p.num_pairs;
-        const int pair = item - bh * p.num_pairs;
-        bool ok = true;
-        if (kside) {  // query tile of the item (the previous item's S MMAs must be done)
-          if (seq > 0 && !wait(&ctl.q_empty, (seq - 1) & 1, kPrKQEmpty)) break;
+      uint32_t qseq = 0;   // items with tiles seen (K side loads their Q tiles)
+      for (uint32_t r = 0;; ++r) {
+        if (!ring_get(r, kside ? kPrKDesc : kPrVDesc)) break;
+        const TileDesc& dsc = ctl.ring[r % kRing];
+        const int flags = dsc.flags, ja = dsc.ja, jb = dsc.jb, bh = dsc.bh, pair = dsc.pair;
+        mbar_arrive(&ctl.ring_empty[r % kRing]);
+        if (flags & kDescEnd) break;
+        if (flags & kDescEmpty) continue;
+        if (kside && (flags & kDescFirst)) {  // the item's query tile (the previous item's S MMAs must be done)
+          if (qseq > 0 && !wait(&ctl.q_empty, (qseq - 1) & 1, kPrKQEmpty)) break;
           mbar_arrive_expect_tx(&ctl.q_full, 128u * D * 2u);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_3d(sQ + cb * CB, &tm_q, &ctl.q_full, cb * 64, 128 * pair, bh);
+          ++qseq;
         }
-        TileIter it;
-        it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
-        Tile t;
-        while (it.next(t)) {
-          uint64_t* empty = kside ? &ctl.k_empty[stage] : &ctl.v_empty[stage];
-          uint64_t* full = kside ? &ctl.k_full[stage] : &ctl.v_full[stage];
-          if (!wait(empty, phase ^ 1u, kside ? kPrKEmpty : kPrVEmpty)) { ok = false; break; }
-          uint8_t* dst = (kside ? sK : sV) + stage * kTile;
-          if (t.kind == 0) {
-            mbar_arrive_expect_tx(full, (kside ? 2u : 1u) * p.W * D * 2u);
+        uint64_t* empty = kside ? &ctl.k_empty[stage] : &ctl.v_empty[stage];
+        uint64_t* full = kside ? &ctl.k_full[stage] : &ctl.v_full[stage];
+        if (!wait(empty, phase ^ 1u, kside ? kPrKEmpty : kPrVEmpty)) break;
+        uint8_t* dst = (kside ? sK : sV) + stage * kTile;
+        if (flags & kDescApprox) {
+          mbar_arrive_expect_tx(full, (kside ? 2u : 1u) * p.W * D * 2u);
 #pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb) {
-              if (kside) {
-                tma_load_3d(dst + cb * CB, &tm_kb, full, cb * 64, t.ja, bh);
-                tma_load_3d(dst + cb * CB + 8192, &tm_kl, full, cb * 64, t.ja, bh);
-              } else {
-                tma_load_3d(dst + cb * CB, &tm_vb, full, cb * 64, t.ja, bh);
-              }
-            }
-          } else {
-            const int nblk = (t.jb >= 0) ? 2 : 1;
-            mbar_arrive_expect_tx(full, static_cast<uint32_t>(nblk) * 64u * D * 2u);
-            const CUtensorMap* map = kside ? &tm_k : &tm_v;
-#pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb) {
-              tma_load_3d(dst + cb * CB, map, full, cb * 64, 64 * t.ja, bh);
-              if (nblk == 2) tma_load_3d(dst + cb * CB + 8192, map, full, cb * 64, 64 * t.jb, bh);
+          for (int cb = 0; cb < D / 64; ++cb) {
+            if (kside) {
+              tma_load_3d(dst + cb * CB, &tm_kb, full, cb * 64, ja, bh);
+              tma_load_3d(dst + cb * CB + 8192, &tm_kl, full, cb * 64, ja, bh);
+            } else {
+              tma_load_3d(dst + cb * CB, &tm_vb, full, cb * 64, ja, bh);
             }
           }
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+        } else {
+          const int nblk = (jb >= 0) ? 2 : 1;
+          mbar_arrive_expect_tx(full, static_cast<uint32_t>(nblk) * 64u * D * 2u);
+          const CUtensorMap* map = kside ? &tm_k : &tm_v;
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb) {
+            tma_load_3d(dst + cb * CB, map, full, cb * 64, 64 * ja, bh);
+            if (nblk == 2) tma_load_3d(dst + cb * CB + 8192, map, full, cb * 64, 64 * jb, bh);
           }
         }
-        mbar_arrive(&ctl.item_empty[s]);
-        if (!ok) break;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
     }
   } else if (warp == 9) {
     // =========================================================== MMA issuer
     if (lane == 0) {
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
       int kstage = 0, vstage = 0;
       uint32_t kphase = 0, vphase = 0;
-      uint32_t tcount = 0;   // tiles whose S MMA is issued (S buffer = index & 1)
-      bool pend = false;     // the PV of tile pv_idx is still to be issued
-      Tile pt{};
-      uint32_t pv_idx = 0;
-      int pv_stage = 0;
-      uint32_t pv_phase = 0;
+      uint32_t tcount = 0;           // tiles whose S MMA is issued; tile t belongs to warpgroup t & 1
+      uint32_t wc0 = 0, wc1 = 0;     // tiles issued per warpgroup
+      uint32_t qseq = 0;             // items with tiles seen
+      bool seen0 = false, seen1 = false;   // warpgroup already had a tile in the current item
+      bool pend = false;             // the PV of the previous tile is still to be issued
+      int pv_ncols = 0, pv_w = 0, pv_stage = 0;
+      uint32_t pv_k = 0, pv_phase = 0;
+      bool pv_first = false;
       bool ok = true;
-      // O (+)= P · Vside for the pending tile.
+      // O_w (+)= P_w · Vside for the pending tile (P_w read from TMEM).
       auto issue_pv = [&]() -> bool {
-        if (!wait(&ctl.p_full, pv_idx & 1, kPrMmaP)) return false;
+        if (!wait(&ctl.p_full[pv_w], pv_k & 1, kPrMmaP)) return false;
         if (!wait(&ctl.v_full[pv_stage], pv_phase, kPrMmaV)) return false;
         tc_fence_after();
-        const int ksteps = pt.ncols / 16;
+        const int ksteps = pv_ncols / 16;
         const uint32_t vbase = sVa + pv_stage * kTile;
-        for (int kk = 0; kk < ksteps; ++kk) {
-          const uint32_t poff = (kk >> 2) * CB + (kk & 3) * 32;
-          umma_ss(tmem + kTmemO, sdesc_sw128(sPa + poff, 16, 1024), sdesc_sw128(vbase + kk * 2048, CB, 1024),
-                  idesc_pv, (pt.first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(&ctl.o_done);
+        const uint32_t pbase = tmem + kTmemS0 + 128 * pv_w;
+        const uint32_t dO = tmem + kTmemO0 + 128 * pv_w;
+        for (int kk = 0; kk < ksteps; ++kk)
+          umma_ts(dO, pbase + 8 * kk, sdesc_sw128(vbase + kk * 2048, CB, 1024), idesc_pv,
+                  (pv_first && kk == 0) ? 0u : 1u);
+        umma_commit(&ctl.o_done[pv_w]);
         umma_commit(&ctl.v_empty[pv_stage]);
         pend = false;
         return true;
       };
-      for (int seq = 0;; ++seq) {
-        const int s = seq & 1;
-        if (!wait(&ctl.item_full[s], (seq >> 1) & 1, kPrMmaItem)) { ok = false; break; }
-        const ItemSlot& sl = ctl.slot[s];
-        const int item = sl.item;
-        if (item < 0) break;
-        const int pair = item % p.num_pairs;
-        if (!wait(&ctl.q_full, seq & 1, kPrMmaQ)) { ok = false; break; }
-        TileIter it;
-        it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
-        Tile t;
-        while (it.next(t)) {
-          // S(t) = Q · Kside^T into S buffer (tcount & 1)
-          const int b = tcount & 1;
-          if (tcount >= 2 && !wait(&ctl.s_empty[b], ((tcount >> 1) - 1) & 1, kPrMmaSEmpty)) { ok = false; break; }
-          if (!wait(&ctl.k_full[kstage], kphase, kPrMmaK)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t dS = tmem + kTmemS0 + b * 128;
-          const uint32_t kbase = sKa + kstage * kTile;
-          const uint32_t idesc_s = idesc_bf16_f32(128, t.ncols, 0);
+      for (uint32_t r = 0;; ++r) {
+        if (!ring_get(r, kPrMmaDesc)) { ok = false; break; }
+        const TileDesc& dsc = ctl.ring[r % kRing];
+        const int flags = dsc.flags, ncols = dsc.ncols;
+        mbar_arrive(&ctl.ring_empty[r % kRing]);
+        if (flags & kDescEnd) break;
+        if (flags & kDescEmpty) continue;
+        if (flags & kDescFirst) {
+          seen0 = seen1 = false;
+          if (!wait(&ctl.q_full, qseq & 1, kPrMmaQ)) { ok = false; break; }
+        }
+        const int w = tcount & 1;
+        const uint32_t k = w ? wc1 : wc0;
+        // S_w / P_w is free once the PV of this warpgroup's previous tile is done
+        if (k >= 1 && !wait(&ctl.o_done[w], (k - 1) & 1, kPrMmaSEmpty)) { ok = false; break; }
+        if (!wait(&ctl.k_full[kstage], kphase, kPrMmaK)) { ok = false; break; }
+        tc_fence_after();
+        // S(t) = Q · Kside^T into S_w
+        const uint32_t dS = tmem + kTmemS0 + 128 * w;
+        const uint32_t kbase = sKa + kstage * kTile;
+        const uint32_t idesc_s = idesc_bf16_f32(128, ncols, 0);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          const uint32_t koff = (kk >> 2) * CB + (kk & 3) * 32;
+          umma_ss(dS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(kbase + koff, 16, 1024), idesc_s,
+                  kk > 0 ? 1u : 0u);
+        }
+        if (flags & kDescApprox) {  // + Q · K̄_lo^T (rows 64.. of the K-side tile)
 #pragma unroll
           for (int kk = 0; kk < KSTEPS; ++kk) {
             const uint32_t koff = (kk >> 2) * CB + (kk & 3) * 32;
-            umma_ss(dS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(kbase + koff, 16, 1024), idesc_s,
-                    kk > 0 ? 1u : 0u);
+            umma_ss(dS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(kbase + 8192 + koff, 16, 1024),
+                    idesc_s, 1u);
           }
-          if (t.kind == 0) {  // + Q · K̄_lo^T (rows 64.. of the K-side tile)
-#pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk) {
-              const uint32_t koff = (kk >> 2) * CB + (kk & 3) * 32;
-              umma_ss(dS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(kbase + 8192 + koff, 16, 1024),
-                      idesc_s, 1u);
-            }
-          }
-          umma_commit(&ctl.s_full[b]);
-          umma_commit(&ctl.k_empty[kstage]);
-          if (++kstage == kStages) {
-            kstage = 0;
-            kphase ^= 1u;
-          }
-          // PV of the previous tile, now that S(t) is queued ahead of it
-          if (pend && !issue_pv()) { ok = false; break; }
-          pt = t;
-          pend = true;
-          pv_idx = tcount;
-          pv_stage = vstage;
-          pv_phase = vphase;
-          if (++vstage == kStages) {
-            vstage = 0;
-            vphase ^= 1u;
-          }
-          ++tcount;
         }
-        if (!ok) break;
-        // every S MMA of this item is issued: Q is free once they complete
-        umma_commit(&ctl.q_empty);
-        mbar_arrive(&ctl.item_empty[s]);
+        umma_commit(&ctl.s_full[w]);
+        umma_commit(&ctl.k_empty[kstage]);
+        if (++kstage == kStages) {
+          kstage = 0;
+          kphase ^= 1u;
+        }
+        if (flags & kDescLast) {  // every S MMA of this item is issued: Q is free once they complete
+          umma_commit(&ctl.q_empty);
+          ++qseq;
+        }
+        // PV of the previous tile, now that S(t) is queued ahead of it
+        if (pend && !issue_pv()) { ok = false; break; }
+        pend = true;
+        pv_ncols = ncols;
+        pv_w = w;
+        pv_k = k;
+        pv_first = w ? !seen1 : !seen0;
+        if (w) seen1 = true; else seen0 = true;
+        pv_stage = vstage;
+        pv_phase = vphase;
+        if (++vstage == kStages) {
+          vstage = 0;
+          vphase ^= 1u;
+        }
+        if (w) wc1 = k + 1; else wc0 = k + 1;
+        ++tcount;
       }
       if (ok && pend) issue_pv();
     }
   } else {
     // =========================================================== softmax (warps 0-7)
-    // Two warpgroups share every tile row: warpgroup wg owns half of the
-    // tile's 32-column groups (and half of O's columns).  Partial row maxima
-    // and, at the end of an item, partial row sums are exchanged through
-    // shared memory behind a bounded mbarrier.
+    // Warpgroup wg handles the tiles of parity wg, one thread per tile row
+    // and all of the row's columns; it keeps its own running max m, sum l and
+    // accumulator O_wg.  The two warpgroups meet once per item to merge.
     const int wg = warp >> 2;
     const int row = tid & 127;        // tile row = TMEM lane
     const int half = row >> 6;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tO = tmem + kTmemO + lane_base;
-    const int tail_n = p.L - 64 * (p.N - 1);
-    constexpr int OG = D / 64;        // 32-column groups of O per warpgroup
-    uint32_t tcount = 0;     // tiles processed
-    uint32_t pv_seen = 0;    // PV completions waited for
+    const uint32_t tS = tmem + kTmemS0 + 128 * wg + lane_base;
+    const uint32_t tO_own = tmem + kTmemO0 + 128 * wg + lane_base;
+    constexpr int OGRP = D / 32;      // 32-column groups of O
+    uint32_t tcount = 0;     // tiles seen (both parities)
+    uint32_t kown = 0;       // own tiles processed
     uint32_t xc = 0;         // exchanges done
-    // Exchange one value per row with the other warpgroup; returns the other's.
-    auto exchange = [&](float v) -> float {
+    // Exchange two values per row with the other warpgroup.
+    auto exchange = [&](float a, float b2, float& oa, float& ob) {
       const int ph = xc & 1;
-      ctl.xval[ph][wg][row] = v;
+      ctl.xval[ph][wg][0][row] = a;
+      ctl.xval[ph][wg][1][row] = b2;
       mbar_arrive(&ctl.xchg);
       wait(&ctl.xchg, ph, kPrSmX);
       ++xc;
-      return ctl.xval[ph][wg ^ 1][row];
+      oa = ctl.xval[ph][wg ^ 1][0][row];
+      ob = ctl.xval[ph][wg ^ 1][1][row];
     };
-    for (int seq = 0;; ++seq) {
-      const int s = seq & 1;
-      if (!wait(&ctl.item_full[s], (seq >> 1) & 1, kPrSmItem)) break;
-      const ItemSlot& sl = ctl.slot[s];
-      const int item = sl.item;
-      if (item < 0) break;
-      const int bh = item / p.num_pairs;
-      const int pair = item - bh * p.num_pairs;
-      const uint32_t* own = sl.mask[half];
-      const int NW = (p.N + 31) >> 5;
-      float m_run = -INFINITY, l_run = 0.f;
-      bool any_tile = false;
-      TileIter it;
-      it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
-      Tile t;
-      // After a timeout every wait returns at once; the loop still runs its
-      // (bounded) course so both warpgroups keep making the same calls.
-      while (it.next(t)) {
-        any_tile = true;
-        const int b = tcount & 1;
-        wait(&ctl.s_full[b], (tcount >> 1) & 1, kPrSmS);
-        tc_fence_after();
-        const uint32_t tS = tmem + kTmemS0 + b * 128 + lane_base;
-        // this warpgroup's 32-column groups of the tile
-        const int ng = t.ncols >> 5;
-        const int gper = (ng >= 2) ? (ng >> 1) : 1;
-        const int g0 = (ng >= 2) ? wg * gper : wg;
-        const int g1 = min(g0 + gper, ng);
-        // validity of a group's 32 columns (warp-uniform: a warp's rows share a half)
-        auto group_bits = [&](int g) -> uint32_t {
-          const int c0 = 32 * g;
-          if (t.kind == 0) {
-            const int nv = min(max(t.avalid - c0, 0), 32);
-            const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
-            return range & ~mask_bits32(own, t.ja + c0, NW);
-          }
-          const int jx = (g < 2) ? t.ja : t.jb;
-          const int key0 = 64 * jx + 32 * (g & 1);
-          const int nv = min(max(p.L - key0, 0), 32);
-          const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
-          return mask_bit(own, jx) ? range : 0u;
-        };
-        SA_PROF(unsigned long long tph = clock64(); prof[kPrSmTiles] += 1;)
-        // Pass 1 reads this thread's 32-column groups from TMEM for the row
-        // maximum; pass 2 reads them again for the probabilities.  Both passes
-        // are runtime loops over one copy of the group code, which keeps the
-        // softmax loop small enough to stay in the instruction cache.
-        // Column adjustments of a group, applied only when needed: invalid
-        // columns become -inf, and the ragged last block's approximation
-        // column gets log2(tail_n / 64) added (its weight is tail_n, not 64).
-        const int tail_col = (t.kind == 0 && tail_n != 64) ? (p.N - 1 - t.ja) : -1;
-        const int tail_g = (tail_col >= 0 && tail_col < t.ncols) ? (tail_col >> 5) : -1;
-        const float tail_raw = (log2f(static_cast<float>(tail_n)) - 6.f) / p.scale_log2;
-        auto adjust = [&](float (&xv)[32], int g) {
-          const uint32_t bits = group_bits(g);
-          const int et = (g == tail_g) ? (tail_col & 31) : -1;
-          if (bits != 0xFFFFFFFFu || et >= 0) {
+    float m_run = -INFINITY, l_run = 0.f;
+    bool own_any = false;    // this warpgroup had a tile in the current item
+    for (uint32_t r = 0;; ++r) {
+      if (!ring_get(r, kPrSmDesc)) break;
+      const TileDesc& dsc = ctl.ring[r % kRing];
+      const uint4 bw = *reinterpret_cast<const uint4*>(dsc.bits[half]);
+      const int ncols = dsc.ncols, dflags = dsc.flags, tail_col = dsc.tail, dbh = dsc.bh, dpair = dsc.pair;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.ring_empty[r % kRing]);
+      if (dflags & kDescEnd) break;
+      if (!(dflags & kDescEmpty)) {
+        const bool mine = (tcount & 1) == static_cast<uint32_t>(wg);
+        ++tcount;
+        if (mine) {
+          wait(&ctl.s_full[wg], kown & 1, kPrSmS);
+          tc_fence_after();
+          SA_PROF(unsigned long long tph = clock64(); prof[kPrSmTiles] += 1;)
+          const int ng = ncols >> 5;   // 32-column groups: 1, 2 or 4
+          auto gb = [&](int i) -> uint32_t { return i == 0 ? bw.x : i == 1 ? bw.y : i == 2 ? bw.z : bw.w; };
+          // Column adjustments, only where needed: invalid columns become -inf,
+          // the ragged block's approximation column gets log2(n_tail / 64).
+          const int tail_g = tail_col >= 0 ? (tail_col >> 5) : -1;
+          auto adjust = [&](float* xv, int g) {
+            const uint32_t bits = gb(g);
+            const int et = (g == tail_g) ? (tail_col & 31) : -1;
+            if (bits != 0xFFFFFFFFu || et >= 0) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (e == et) xv[e] += tail_raw;
-              if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
+              for (int e = 0; e < 32; ++e) {
+                if (e == et) xv[e] += p.tail_raw;
+                if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
+              }
+            }
+          };
+          // pass 1: row maximum, two groups per TMEM round trip
+          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll 1
+          for (int g = 0; g < ng; g += 2) {
+            float xv[64];
+            tmem_ld_x32f(tS + 32 * g, xv);
+            if (g + 1 < ng) tmem_ld_x32f(tS + 32 * (g + 1), xv + 32);
+            tmem_ld_wait();
+            reg_fence32(xv);
+            reg_fence32(xv + 32);
+            adjust(xv, g);
+            if (g + 1 < ng) {
+              adjust(xv + 32, g + 1);
+            } else {
+#pragma unroll
+              for (int e = 32; e < 64; ++e) xv[e] = -INFINITY;
+            }
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              mx0 = max3f(mx0, xv[e], xv[e + 1]);
+              mx1 = max3f(mx1, xv[e + 2], xv[e + 3]);
+              mx2 = max3f(mx2, xv[e + 32], xv[e + 33]);
+              mx3 = max3f(mx3, xv[e + 34], xv[e + 35]);
             }
           }
-        };
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll 1
-        for (int g = g0; g < g1; ++g) {
-          float xv[32];
-          tmem_ld_x32f(tS + 32 * g, xv);
-          tmem_ld_wait();
-          reg_fence32(xv);
-          adjust(xv, g);
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            mx0 = max3f(mx0, xv[e], xv[e + 1]);
-            mx1 = max3f(mx1, xv[e + 2], xv[e + 3]);
-            mx2 = max3f(mx2, xv[e + 4], xv[e + 5]);
-            mx3 = max3f(mx3, xv[e + 6], xv[e + 7]);
+          const float rmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+          SA_PROF(prof[kPrSmPass1] += clock64() - tph; tph = clock64();)
+          // In log2 units.  An approximation column stands for its n_j tokens:
+          // its weight n_j is folded into the logit as + log2(n_j) (6 for a full
+          // block) and the value side uses the block mean V̂_j / n_j.
+          const float boost = (dflags & kDescApprox) ? 6.f : 0.f;
+          const float tmax = (rmax == -INFINITY) ? -INFINITY : fmaf(rmax, p.scale_log2, boost);
+          // lazy rescale: move the reference max only when it grows by > 8 (x256)
+          const bool first_own = !own_any;
+          if (first_own) {
+            m_run = -INFINITY;
+            l_run = 0.f;
           }
-        }
-        const float pmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-        SA_PROF(prof[kPrSmPass1] += clock64() - tph;)
-        const float rmax = fmaxf(pmax, exchange(pmax));
-        // In log2 units.  An approximation column stands for its n_j tokens:
-        // its weight n_j is folded into the logit as + log2(n_j) (6 for a full
-        // block) and the value side uses the block mean V̂_j / n_j.
-        const float boost = (t.kind == 0) ? 6.f : 0.f;
-        const float tmax = (rmax == -INFINITY) ? -INFINITY : fmaf(rmax, p.scale_log2, boost);
-        // lazy rescale: move the reference max only when it grows by > 8 (x256);
-        // both warpgroups take the same decision from the same row maximum
-        const bool need = tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY);
-        float alpha = 1.f;
-        if (need) {
-          const float m_new = fmaxf(m_run, tmax);
-          alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
-          l_run *= alpha;
-          m_run = m_new;
-        }
-        const float off = boost - ((m_run == -INFINITY) ? 0.f : m_run);
-        // the previous tile's PV must be done before P is overwritten or O rescaled
-        if (pv_seen < tcount) {
-          wait(&ctl.o_done, (tcount - 1) & 1, kPrSmO);
-          pv_seen = tcount;
-          tc_fence_after();
-        }
-        SA_PROF(tph = clock64();)
-        if (!t.first && __any_sync(0xFFFFFFFFu, need)) {
-          SA_PROF(prof[kPrSmRescales] += 1;)
+          const bool need = tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY);
+          float alpha = 1.f;
+          if (need) {
+            const float m_new = fmaxf(m_run, tmax);
+            alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
+            l_run *= alpha;
+            m_run = m_new;
+          }
+          const float off = boost - ((m_run == -INFINITY) ? 0.f : m_run);
+          // O_wg holds this warpgroup's previous tiles; their PVs completed before
+          // the MMA issuer wrote this S tile (it waits for them), so O_wg is stable.
+          if (!first_own && __any_sync(0xFFFFFFFFu, need)) {
+            SA_PROF(prof[kPrSmRescales] += 1;)
 #pragma unroll 1
-          for (int c32 = wg * OG; c32 < (wg + 1) * OG; ++c32) {
-            uint32_t r[32];
-            tmem_ld_x32(tO + c32 * 32, r);
+            for (int c32 = 0; c32 < OGRP; ++c32) {
+              uint32_t rr[32];
+              tmem_ld_x32(tO_own + c32 * 32, rr);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+              tmem_st_x32(tO_own + c32 * 32, rr);
+            }
+          }
+          SA_PROF(prof[kPrSmRescale] += clock64() - tph; tph = clock64();)
+          // pass 2: probabilities and row sum; P goes back into TMEM over S
+          // (bf16 pairs, 16 columns per 32 probabilities) as the PV MMA's A.
+          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+          const float2 of2 = make_float2(off, off);
+          float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+#pragma unroll 1
+          for (int g = 0; g < ng; ++g) {
+            float xv[32];
+            tmem_ld_x32f(tS + 32 * g, xv);
             tmem_ld_wait();
+            reg_fence32(xv);
+            adjust(xv, g);
+            uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st_x32(tO + c32 * 32, r);
+            for (int e = 0; e < 32; e += 8) {
+              const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
+              const float2 y1 = __ffma2_rn(make_float2(xv[e + 2], xv[e + 3]), sc2, of2);
+              const float2 y2 = __ffma2_rn(make_float2(xv[e + 4], xv[e + 5]), sc2, of2);
+              const float2 y3 = __ffma2_rn(make_float2(xv[e + 6], xv[e + 7]), sc2, of2);
+              const float2 q0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+              const float2 q1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+              const float2 q2 = make_float2(ex2_approx(y2.x), ex2_approx(y2.y));
+              const float2 q3 = make_float2(ex2_approx(y3.x), ex2_approx(y3.y));
+              sa = __fadd2_rn(sa, __fadd2_rn(q0, q2));
+              sb = __fadd2_rn(sb, __fadd2_rn(q1, q3));
+              pk[e >> 1] = pack_bf16x2(q0.x, q0.y);
+              pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
+              pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
+              pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
+            }
+            // P of group g lands in columns [16g, 16g+16), inside S groups that
+            // were already read (this pass reads group g before writing it)
+            tmem_st_x16(tS + 16 * g, pk);
           }
+          l_run += (sa.x + sa.y) + (sb.x + sb.y);
           tmem_st_wait();
+          SA_PROF(prof[kPrSmPass2] += clock64() - tph;)
+          tc_fence_before();
+          mbar_arrive(&ctl.p_full[wg]);
+          ++kown;
+          own_any = true;
         }
-        SA_PROF(prof[kPrSmRescale] += clock64() - tph; tph = clock64();)
-        // pass 2: probabilities, partial row sum, P to shared memory.  12 of
-        // every 32 exponentials run on the FMA/ALU pipes (exp2_poly), the rest
-        // on MUFU; masked columns hold -inf and give 0 either way.
-        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-        const float2 of2 = make_float2(off, off);
-        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-#pragma unroll 1
-        for (int g = g0; g < g1; ++g) {
-          float xv[32];
-          tmem_ld_x32f(tS + 32 * g, xv);
-          tmem_ld_wait();
-          reg_fence32(xv);
-          adjust(xv, g);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
-            const float2 y1 = __ffma2_rn(make_float2(xv[e + 2], xv[e + 3]), sc2, of2);
-            const float2 y2 = __ffma2_rn(make_float2(xv[e + 4], xv[e + 5]), sc2, of2);
-            const float2 y3 = __ffma2_rn(make_float2(xv[e + 6], xv[e + 7]), sc2, of2);
-            const float2 q0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
-            const float2 q1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
-            const float2 q2 = make_float2(ex2_approx(y2.x), exp2_poly(y2.y));
-            const float2 q3 = make_float2(exp2_poly(y3.x), exp2_poly(y3.y));
-            sa = __fadd2_rn(sa, __fadd2_rn(q0, q2));
-            sb = __fadd2_rn(sb, __fadd2_rn(q1, q3));
-            pk[e >> 1] = pack_bf16x2(q0.x, q0.y);
-            pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
-            pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
-            pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
-          }
-          store_p32(sP, row, 32 * g, pk);
-        }
-        l_run += (sa.x + sa.y) + (sb.x + sb.y);
-        SA_PROF(prof[kPrSmPass2] += clock64() - tph;)
-        // S buffer b may now be overwritten by the MMA of tile tcount + 2
-        tc_fence_before();
-        mbar_arrive(&ctl.s_empty[b]);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&ctl.p_full);
-        ++tcount;
       }
-      // ---- epilogue: row sum of both warpgroups, last PV, O / l for rows < L (Eq. 10)
+      if (!(dflags & (kDescLast | kDescEmpty))) continue;
+      // ---- epilogue: merge the two warpgroups' partial softmaxes (Eq. 10)
       SA_PROF(const unsigned long long tep = clock64();)
-      const float l_tot = l_run + exchange(l_run);
-      if (tcount > pv_seen) {
-        wait(&ctl.o_done, (tcount - 1) & 1, kPrSmO);
-        pv_seen = tcount;
+      if (own_any) {   // this warpgroup's last PV
+        wait(&ctl.o_done[wg], (kown - 1) & 1, kPrSmO);
         tc_fence_after();
       }
-      const int token = 128 * pair + row;
+      const float my_m = own_any ? m_run : -INFINITY;
+      const float my_l = own_any ? l_run : 0.f;
+      float ot_m, ot_l;
+      exchange(my_m, my_l, ot_m, ot_l);
+      tc_fence_after();
+      const float mm = fmaxf(my_m, ot_m);
+      const float f_own = (my_m == -INFINITY) ? 0.f : ex2_approx(my_m - mm);
+      const float f_oth = (ot_m == -INFINITY) ? 0.f : ex2_approx(ot_m - mm);
+      const float l_tot = f_own * my_l + f_oth * ot_l;
       const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
-      uint16_t* orow = p.out + (static_cast<size_t>(bh) * p.L + token) * D;
+      const float w_own = f_own * inv_l, w_oth = f_oth * inv_l;
+      const bool own_has = own_any && w_own != 0.f, oth_has = (ot_m != -INFINITY) && w_oth != 0.f;
+      const int token = 128 * dpair + row;
+      uint16_t* orow = p.out + (static_cast<size_t>(dbh) * p.L + token) * D;
+      // warpgroup wg writes O columns [wg * D/2, (wg + 1) * D/2), 16 at a time
 #pragma unroll 1
-      for (int c32 = wg * OG; c32 < (wg + 1) * OG; ++c32) {
-        uint32_t r[32];
-        if (any_tile) {            // an item with no tile (exact-only, nothing selected) outputs 0
-          tmem_ld_x32(tO + c32 * 32, r);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = 0u;
-        }
+      for (int c16 = wg * D / 32; c16 < (wg + 1) * D / 32; ++c16) {
+        float a[16], c[16];
+        if (own_has) tmem_ld_x16f(tmem + kTmemO0 + 128 * wg + lane_base + c16 * 16, a);
+        if (oth_has) tmem_ld_x16f(tmem + kTmemO0 + 128 * (wg ^ 1) + lane_base + c16 * 16, c);
+        tmem_ld_wait();
+        reg_fence16(a);
+        reg_fence16(c);
         if (token < p.L) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]) * inv_l, __uint_as_float(r[8 * g + 1]) * inv_l);
-            v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]) * inv_l, __uint_as_float(r[8 * g + 3]) * inv_l);
-            v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]) * inv_l, __uint_as_float(r[8 * g + 5]) * inv_l);
-            v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]) * inv_l, __uint_as_float(r[8 * g + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(orow + c32 * 32 + 8 * g) = v;
-          }
+          for (int e = 0; e < 16; ++e)
+            a[e] = (own_has ? a[e] * w_own : 0.f) + (oth_has ? c[e] * w_oth : 0.f);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c16 * 16);
+          dst[0] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                              pack_bf16x2(a[6], a[7]));
+          dst[1] = make_uint4(pack_bf16x2(a[8], a[9]), pack_bf16x2(a[10], a[11]), pack_bf16x2(a[12], a[13]),
+                              pack_bf16x2(a[14], a[15]));
         }
       }
-      SA_PROF(prof[kPrSmEpi] += clock64() - tep;)
+      // both warpgroups are done reading O_0 and O_1 before either can start
+      // the next item (whose first PVs overwrite them)
       tc_fence_before();
-      mbar_arrive(&ctl.item_empty[s]);
+      float d0, d1;
+      exchange(0.f, 0.f, d0, d1);
+      own_any = false;
+      SA_PROF(prof[kPrSmEpi] += clock64() - tep;)
     }
   }
 
   SA_PROF({
-    const int tslot = warp == 11 ? kPrTotRoute : warp == 8 ? kPrTotK : warp == 10 ? kPrTotV
-                    : warp == 9 ? kPrTotMma : kPrTotSm;
-    if (lane == 0 && (warp >= 8 || warp == 0)) {
+    const int tslot = warp == 10 ? kPrTotRoute : warp == 11 ? kPrTotSched : warp == 9 ? kPrTotMma
+                    : warp == 8 ? (lane == 0 ? kPrTotK : kPrTotV) : kPrTotSm;
+    if ((lane == 0 && (warp >= 8 || warp == 0)) || (warp == 8 && lane == 1)) {
       prof[tslot] = clock64() - prof_t0;
       for (int i = 0; i < kPrSlots; ++i) if (prof[i]) atomicAdd(&g_profile[i], prof[i]);
     }

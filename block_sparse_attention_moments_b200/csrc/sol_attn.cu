@@ -301,6 +301,10 @@ int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void
   p.flags = flags;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   p.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  {
+    const int tail_n = s.L - 64 * (N - 1);
+    p.tail_raw = static_cast<float>((std::log2(static_cast<double>(tail_n)) - 6.0) / static_cast<double>(p.scale_log2));
+  }
   p.qbar = w.qbar;
   p.kbar = w.kbar;
   p.tau = w.tau;
