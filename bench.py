@@ -124,11 +124,17 @@ def dist_setup(n_gpus: int):
     return rank, world, local, pg
 
 
+def _reduce_device(pg):
+    """NCCL reduces CUDA tensors; gloo (CPU tests of this path) reduces host tensors."""
+    return "cuda" if pg.get_backend() == "nccl" else "cpu"
+
+
 def max_over_ranks(x: float, pg) -> float:
+    """Timing of a multi-GPU step: the slowest rank's (host-side reduction, not a data-path collective)."""
     if pg is None:
         return x
     import torch
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=_reduce_device(pg), dtype=torch.float64)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
 
@@ -137,9 +143,18 @@ def sum_over_ranks(x: float, pg) -> float:
     if pg is None:
         return x
     import torch
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=_reduce_device(pg), dtype=torch.float64)
     pg.all_reduce(t, op=pg.ReduceOp.SUM)
     return float(t.item())
+
+
+WORKLOAD_TEXT = {
+    "tiny": "tiny check B=1 H=1 L=1024 (4x16x16) d=64",
+    "small": "small B=1 H=2 L=4096 (4x32x32) d=128",
+    "image": "image-generation shape B=2 H=24 L=16384 (1x128x128) d=128",
+    "wan": "Wan-2.1-14B-like self-attention B=1 H=40 L=75600 (21x45x80) d=128",
+    "hunyuan": "HunyuanVideo-13B-like self-attention B=1 H=24 L=118800 (33x45x80) d=128",
+}
 
 
 def rank_inputs(wl, rank: int):
@@ -379,8 +394,8 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"{wl.name}: Wan-2.1-14B-like self-attention B=1 H={H} L={L} (21x45x80) d={d} "
-                               f"block=64 C={C} beta={args.beta}, bf16 Fourier-feature Q/K, Gaussian V",
+        "config": {"workload": f"{wl.name}: {WORKLOAD_TEXT.get(wl.name, wl.name)} per GPU, block=64 C={C} "
+                               f"beta={args.beta}, bf16 Fourier-feature Q/K, Gaussian V",
                    "per_gpu_batch": 1, "global_batch": world, "seq_len": L, "parallelism": f"dp{world} (weak)",
                    "l2": "inputs (2.3 GB/step) larger than L2 (126 MB)"},
         "ms_per_call": step_ms,
