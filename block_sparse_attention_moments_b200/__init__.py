@@ -226,14 +226,15 @@ PROFILE_SLOTS = (
     "softmax.wait_desc", "softmax.wait_s", "softmax.wait_o", "softmax.wait_exchange",
     "total.route", "total.k", "total.v", "total.mma", "total.softmax",
     "softmax.pass1", "softmax.rescale", "softmax.pass2", "softmax.epilogue", "softmax.tiles", "softmax.rescales",
-    "sched.wait_item", "sched.wait_ring", "total.sched",
+    "sched.wait_item", "sched.wait_ring", "total.sched", "softmax.redos",
+    "mma.issue_s", "mma.issue_pv",
 )
 
 
 def profile_read(reset: bool = True) -> dict:
     """Cycle counters of the profiling build, summed over CTAs (see sol_attn_profile_read)."""
-    buf = (ctypes.c_uint64 * 32)()
-    _check(lib().sol_attn_profile_read(buf, 32, 1 if reset else 0))
+    buf = (ctypes.c_uint64 * 48)()
+    _check(lib().sol_attn_profile_read(buf, 48, 1 if reset else 0))
     return {name: int(buf[k]) for k, name in enumerate(PROFILE_SLOTS)}
 
 

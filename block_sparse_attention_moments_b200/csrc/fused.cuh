@@ -74,10 +74,12 @@ enum ProfSlot : int {
   kPrSmDesc, kPrSmS, kPrSmO, kPrSmX,
   kPrTotRoute, kPrTotK, kPrTotV, kPrTotMma, kPrTotSm,
   kPrSmPass1, kPrSmRescale, kPrSmPass2, kPrSmEpi, kPrSmTiles, kPrSmRescales, kPrSchedItem, kPrSchedRing,
-  kPrTotSched, kPrSlots
+  kPrTotSched, kPrSmRedo, kPrMmaIssueS, kPrMmaIssuePV, kPrSlots
 };
+constexpr int kProfileSlots = 48;
+static_assert(kPrSlots <= kProfileSlots, "profile slots");
 #ifdef SOL_ATTN_PROFILE
-__device__ unsigned long long g_profile[32];
+__device__ unsigned long long g_profile[kProfileSlots];
 #define SA_PROF(x) x
 #else
 #define SA_PROF(x)
@@ -180,16 +182,28 @@ struct Tile {
   bool first;  // first tile of its item (PV overwrites O)
 };
 
-// Walks an item's tile sequence: for each chunk, approximation sub-tiles
-// (skipped when both halves selected every block in them), then the union of
-// the selected blocks, two per tile.  Run by the scheduler warp.
+// Walks an item's tile sequence, one chunk of C pooled keys at a time: the
+// union of the selected blocks, two per tile, then the chunk's approximation
+// sub-tiles (skipped when both halves selected every block in them).  The walk
+// starts at the chunk that holds the item's own query blocks, and inside that
+// chunk at block i0, then wraps around.  The online softmax is independent of
+// the order of its tiles up to rounding; starting near the diagonal makes the
+// first tiles carry each row's largest logits, so the running maximum rarely
+// moves afterwards.  Run by the scheduler warp.
 struct TileIter {
   const uint32_t* m0;
   const uint32_t* m1;
-  int N, C, W, nw;
+  int N, C, W;
+  int nw;           // mask words per half
   bool has1, exact_only, first;
-  int lo, hi, a0, j;
+  int lo, hi;       // current chunk [lo, hi)
+  int jstart;       // the chunk's exact blocks run over [jstart, hi) then [lo, jstart)
+  int seg;          // 0, 1: position in those two ranges; 2: exact blocks done
+  int j;            // next candidate block of the current range
+  int a0;           // next approximation sub-tile start
+  int chunks_left;
 
+  // First block of the union of both selections in [from, lim), or lim.
   __device__ __forceinline__ int next_union(int from, int lim) const {
     int x = from;
     while (x < lim) {
@@ -203,12 +217,29 @@ struct TileIter {
     }
     return lim;
   }
-  __device__ __forceinline__ void start_chunk() {
-    hi = min(lo + C, N);
-    a0 = exact_only ? hi : lo;
-    j = next_union(lo, hi);
+  // Next selected block of the current chunk in its exact order, or -1.
+  __device__ __forceinline__ int next_exact() {
+    while (seg < 2) {
+      const int lim = seg == 0 ? hi : jstart;
+      const int jj = next_union(j, lim);
+      if (jj < lim) {
+        j = jj + 1;
+        return jj;
+      }
+      ++seg;
+      j = lo;
+    }
+    return -1;
   }
-  __device__ __forceinline__ void init(const ItemSlot& s, int N_, int C_, int W_, bool has1_, bool exact_only_) {
+  __device__ __forceinline__ void start_chunk(int start) {
+    hi = min(lo + C, N);
+    jstart = start;
+    seg = 0;
+    j = start;
+    a0 = exact_only ? hi : lo;
+  }
+  __device__ __forceinline__ void init(const ItemSlot& s, int N_, int C_, int W_, int i0, bool has1_,
+                                       bool exact_only_) {
     m0 = s.mask[0];
     m1 = s.mask[1];
     N = N_;
@@ -218,11 +249,19 @@ struct TileIter {
     has1 = has1_;
     exact_only = exact_only_;
     first = true;
-    lo = 0;
-    start_chunk();
+    chunks_left = (N_ + C_ - 1) / C_;
+    lo = (i0 / C_) * C_;
+    start_chunk(i0);
   }
   __device__ __forceinline__ bool next(Tile& t) {
-    while (lo < N) {
+    while (chunks_left > 0) {
+      const int ja = next_exact();
+      if (ja >= 0) {
+        const int jb = next_exact();
+        t = (jb >= 0) ? Tile{1, ja, jb, 128, 0, first} : Tile{1, ja, -1, 64, 0, first};
+        first = false;
+        return true;
+      }
       while (a0 < hi) {
         const int a1 = min(a0 + W, hi);
         const int s = a0;
@@ -241,20 +280,10 @@ struct TileIter {
           return true;
         }
       }
-      if (j < hi) {
-        const int jb = next_union(j + 1, hi);
-        if (jb < hi) {
-          t = Tile{1, j, jb, 128, 0, first};
-          j = next_union(jb + 1, hi);
-        } else {
-          t = Tile{1, j, -1, 64, 0, first};
-          j = hi;
-        }
-        first = false;
-        return true;
+      if (--chunks_left > 0) {
+        lo = (hi >= N) ? 0 : hi;
+        start_chunk(lo);
       }
-      lo = hi;
-      if (lo < N) start_chunk();
     }
     return false;
   }
@@ -450,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         publish();
       } else {
         TileIter it;
-        it.init(sl, p.N, p.chunk, p.W, 2 * pair + 1 < p.N, exact_only);
+        it.init(sl, p.N, p.chunk, p.W, 2 * pair, 2 * pair + 1 < p.N, exact_only);
         Tile t, tn;
         bool have = it.next(t);
         bool first_desc = true;
@@ -568,6 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait(&ctl.p_full[pv_w], pv_k & 1, kPrMmaP)) return false;
         if (!wait(&ctl.v_full[pv_stage], pv_phase, kPrMmaV)) return false;
         tc_fence_after();
+        SA_PROF(const unsigned long long tis = clock64();)
         const int ksteps = pv_ncols / 16;
         const uint32_t vbase = sVa + pv_stage * kTile;
         const uint32_t pbase = tmem + kTmemS0 + 128 * pv_w;
@@ -577,6 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (pv_first && kk == 0) ? 0u : 1u);
         umma_commit(&ctl.o_done[pv_w]);
         umma_commit(&ctl.v_empty[pv_stage]);
+        SA_PROF(prof[kPrMmaIssuePV] += clock64() - tis;)
         pend = false;
         return true;
       };
@@ -597,6 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (k >= 1 && !wait(&ctl.o_done[w], (k - 1) & 1, kPrMmaSEmpty)) { ok = false; break; }
         if (!wait(&ctl.k_full[kstage], kphase, kPrMmaK)) { ok = false; break; }
         tc_fence_after();
+        SA_PROF(const unsigned long long tis = clock64();)
         // S(t) = Q · Kside^T into S_w
         const uint32_t dS = tmem + kTmemS0 + 128 * w;
         const uint32_t kbase = sKa + kstage * kTile;
@@ -617,6 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(&ctl.s_full[w]);
         umma_commit(&ctl.k_empty[kstage]);
+        SA_PROF(prof[kPrMmaIssueS] += clock64() - tis;)
         if (++kstage == kStages) {
           kstage = 0;
           kphase ^= 1u;
@@ -655,7 +688,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + kTmemS0 + 128 * wg + lane_base;
     const uint32_t tO_own = tmem + kTmemO0 + 128 * wg + lane_base;
-    constexpr int OGRP = D / 32;      // 32-column groups of O
     uint32_t tcount = 0;     // tiles seen (both parities)
     uint32_t kown = 0;       // own tiles processed
     uint32_t xc = 0;         // exchanges done
@@ -703,101 +735,139 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           };
-          // pass 1: row maximum, two groups per TMEM round trip
-          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll 1
-          for (int g = 0; g < ng; g += 2) {
-            float xv[64];
-            tmem_ld_x32f(tS + 32 * g, xv);
-            if (g + 1 < ng) tmem_ld_x32f(tS + 32 * (g + 1), xv + 32);
-            tmem_ld_wait();
-            reg_fence32(xv);
-            reg_fence32(xv + 32);
-            adjust(xv, g);
-            if (g + 1 < ng) {
-              adjust(xv + 32, g + 1);
-            } else {
-#pragma unroll
-              for (int e = 32; e < 64; ++e) xv[e] = -INFINITY;
-            }
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              mx0 = max3f(mx0, xv[e], xv[e + 1]);
-              mx1 = max3f(mx1, xv[e + 2], xv[e + 3]);
-              mx2 = max3f(mx2, xv[e + 32], xv[e + 33]);
-              mx3 = max3f(mx3, xv[e + 34], xv[e + 35]);
-            }
-          }
-          const float rmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-          SA_PROF(prof[kPrSmPass1] += clock64() - tph; tph = clock64();)
           // In log2 units.  An approximation column stands for its n_j tokens:
           // its weight n_j is folded into the logit as + log2(n_j) (6 for a full
           // block) and the value side uses the block mean V̂_j / n_j.
           const float boost = (dflags & kDescApprox) ? 6.f : 0.f;
-          const float tmax = (rmax == -INFINITY) ? -INFINITY : fmaf(rmax, p.scale_log2, boost);
-          // lazy rescale: move the reference max only when it grows by > 8 (x256)
           const bool first_own = !own_any;
           if (first_own) {
             m_run = -INFINITY;
             l_run = 0.f;
           }
-          const bool need = tmax > m_run + 8.f || (m_run == -INFINITY && tmax != -INFINITY);
-          float alpha = 1.f;
-          if (need) {
-            const float m_new = fmaxf(m_run, tmax);
-            alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
-            l_run *= alpha;
-            m_run = m_new;
-          }
-          const float off = boost - ((m_run == -INFINITY) ? 0.f : m_run);
-          // O_wg holds this warpgroup's previous tiles; their PVs completed before
-          // the MMA issuer wrote this S tile (it waits for them), so O_wg is stable.
-          if (!first_own && __any_sync(0xFFFFFFFFu, need)) {
-            SA_PROF(prof[kPrSmRescales] += 1;)
-#pragma unroll 1
-            for (int c32 = 0; c32 < OGRP; ++c32) {
-              uint32_t rr[32];
-              tmem_ld_x32(tO_own + c32 * 32, rr);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-              tmem_st_x32(tO_own + c32 * 32, rr);
-            }
-          }
-          SA_PROF(prof[kPrSmRescale] += clock64() - tph; tph = clock64();)
-          // pass 2: probabilities and row sum; P goes back into TMEM over S
-          // (bf16 pairs, 16 columns per 32 probabilities) as the PV MMA's A.
           const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-          const float2 of2 = make_float2(off, off);
           float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-#pragma unroll 1
-          for (int g = 0; g < ng; ++g) {
-            float xv[32];
-            tmem_ld_x32f(tS + 32 * g, xv);
-            tmem_ld_wait();
-            reg_fence32(xv);
-            adjust(xv, g);
-            uint32_t pk[16];
+          // p = 2^y, y = x * scale_log2 + off, for 32 adjusted columns, packed as
+          // 16 bf16 pairs; the fp32 values go into the row sum (ra, rb) and the
+          // largest y into ym.
+          auto probs32 = [&](const float* xv, float2 of2, uint32_t* pk, float2& ra, float2& rb, float& ym) {
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
               const float2 y1 = __ffma2_rn(make_float2(xv[e + 2], xv[e + 3]), sc2, of2);
               const float2 y2 = __ffma2_rn(make_float2(xv[e + 4], xv[e + 5]), sc2, of2);
               const float2 y3 = __ffma2_rn(make_float2(xv[e + 6], xv[e + 7]), sc2, of2);
+              ym = max3f(ym, max3f(y0.x, y0.y, y1.x), max3f(y1.y, y2.x, y2.y));
+              ym = max3f(ym, y3.x, y3.y);
               const float2 q0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
               const float2 q1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
               const float2 q2 = make_float2(ex2_approx(y2.x), ex2_approx(y2.y));
               const float2 q3 = make_float2(ex2_approx(y3.x), ex2_approx(y3.y));
-              sa = __fadd2_rn(sa, __fadd2_rn(q0, q2));
-              sb = __fadd2_rn(sb, __fadd2_rn(q1, q3));
+              ra = __fadd2_rn(ra, __fadd2_rn(q0, q2));
+              rb = __fadd2_rn(rb, __fadd2_rn(q1, q3));
               pk[e >> 1] = pack_bf16x2(q0.x, q0.y);
               pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
               pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
               pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
             }
-            // P of group g lands in columns [16g, 16g+16), inside S groups that
-            // were already read (this pass reads group g before writing it)
-            tmem_st_x16(tS + 16 * g, pk);
+          };
+          // Read, adjust and exponentiate groups g0 and g0 + 1 (those below ng)
+          // into pk[0, 32); returns the largest y.
+          auto half_tile = [&](int g0, float2 of2, uint32_t* pk, float2& ra, float2& rb) -> float {
+            float ym = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (g0 + h < ng) {
+                float xv[32];
+                tmem_ld_x32f(tS + 32 * (g0 + h), xv);
+                tmem_ld_wait();
+                reg_fence32(xv);
+                adjust(xv, g0 + h);
+                probs32(xv, of2, pk + 16 * h, ra, rb, ym);
+              }
+            }
+            return ym;
+          };
+          // O_wg *= alpha (per row).  O_wg holds this warpgroup's previous tiles;
+          // their PVs completed before the MMA issuer wrote this S tile (it waits
+          // for them), so O_wg is stable.
+          auto rescale_o = [&](float alpha) {
+            SA_PROF(prof[kPrSmRescales] += 1;)
+#pragma unroll 1
+            for (int c16 = 0; c16 < D; c16 += 16) {
+              float rr[16];
+              tmem_ld_x16f(tO_own + c16, rr);
+              tmem_ld_wait();
+              reg_fence16(rr);
+              uint32_t pw[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pw[e] = __float_as_uint(rr[e] * alpha);
+              tmem_st_x16(tO_own + c16, pw);
+            }
+          };
+          // One pass over S, 64 columns (a half) at a time, against the current
+          // reference maximum m (0 while the row has seen no valid column).  P
+          // of a half stays in registers until the half's largest y is known:
+          // while every row of the warp has y <= 8 the lazy rescale rule keeps m
+          // and P lands in TMEM as computed.  Otherwise the rows past the limit
+          // raise m (to their maximum on a first valid column, else by a whole
+          // number k of doublings, so that the values already accumulated scale
+          // by 2^-k exactly, even P already in bf16) and the half is recomputed
+          // from S, which no P store has reached yet: half h's P goes to
+          // columns [32h, 32h + 32), over S groups that were read before it.
+          const int nh = (ng + 1) >> 1;
+          int redo = 0;   // recomputations of the current half (one suffices; two bound the loop)
+#pragma unroll 1
+          for (int h = 0; h < nh;) {
+            const float mref = (m_run == -INFINITY) ? 0.f : m_run;
+            const float2 of2 = make_float2(boost - mref, boost - mref);
+            float2 ha = make_float2(0.f, 0.f), hb = make_float2(0.f, 0.f);
+            uint32_t pk[32];
+            const float ym = half_tile(2 * h, of2, pk, ha, hb);
+            const bool ex = (m_run == -INFINITY) ? (ym != -INFINITY) : (ym > 8.f);
+            if (redo < 2 && __any_sync(0xFFFFFFFFu, ex)) {
+              ++redo;
+              SA_PROF(prof[kPrSmRedo] += 1;)
+              float alpha = 1.f;
+              if (ex) {
+                if (m_run == -INFINITY) {
+                  m_run = ym;       // y was measured against 0: this is the maximum itself
+                  alpha = 0.f;      // nothing valid accumulated yet
+                } else {
+                  const float k = ceilf(ym);
+                  m_run += k;
+                  alpha = (k >= 126.f) ? 0.f : __int_as_float((127 - static_cast<int>(k)) << 23);
+                }
+                l_run *= alpha;
+                sa = make_float2(sa.x * alpha, sa.y * alpha);
+                sb = make_float2(sb.x * alpha, sb.y * alpha);
+              }
+              __syncwarp();
+              if (h > 0) {   // P of columns [0, 64), already in TMEM columns [0, 32)
+                tmem_st_wait();
+#pragma unroll 1
+                for (int c16 = 0; c16 < 32; c16 += 16) {
+                  float rr[16];
+                  tmem_ld_x16f(tS + c16, rr);
+                  tmem_ld_wait();
+                  reg_fence16(rr);
+                  uint32_t pw[16];
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) {
+                    const uint32_t u = __float_as_uint(rr[e]);
+                    pw[e] = pack_bf16x2(__uint_as_float(u << 16) * alpha, __uint_as_float(u & 0xFFFF0000u) * alpha);
+                  }
+                  tmem_st_x16(tS + c16, pw);
+                }
+              }
+              if (!first_own) rescale_o(alpha);
+              continue;   // the same half again, against the new m
+            }
+            tmem_st_x16(tS + 32 * h, pk);
+            if (2 * h + 1 < ng) tmem_st_x16(tS + 32 * h + 16, pk + 16);
+            sa = __fadd2_rn(sa, ha);
+            sb = __fadd2_rn(sb, hb);
+            ++h;
+            redo = 0;
           }
           l_run += (sa.x + sa.y) + (sb.x + sb.y);
           tmem_st_wait();

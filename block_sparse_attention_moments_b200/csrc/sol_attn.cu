@@ -567,12 +567,12 @@ int sol_attn_kernels_per_forward(void) { return 4; }
 int sol_attn_profile_read(uint64_t* cycles, int n, int reset) {
 #ifdef SOL_ATTN_PROFILE
   if (!cycles || n < 1) return fail(SOL_ATTN_ERR_ARG, "cycles is NULL or n < 1");
-  unsigned long long h[32];
+  unsigned long long h[kProfileSlots];
   CUDA_TRY(cudaDeviceSynchronize());
   CUDA_TRY(cudaMemcpyFromSymbol(h, g_profile, sizeof(h)));
-  for (int i = 0; i < n && i < 32; ++i) cycles[i] = h[i];
+  for (int i = 0; i < n && i < kProfileSlots; ++i) cycles[i] = h[i];
   if (reset) {
-    unsigned long long z[32] = {0};
+    unsigned long long z[kProfileSlots] = {0};
     CUDA_TRY(cudaMemcpyToSymbol(g_profile, z, sizeof(z)));
   }
   return SOL_ATTN_OK;

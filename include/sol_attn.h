@@ -133,7 +133,7 @@ int sol_attn_kernels_per_forward(void);
 /* Per-role cycle accounting of the fused kernel (tracing aid; no counterpart in
  * the paper).  Only a library built with -DSOL_ATTN_PROFILE (libsol_attn_profile.so)
  * collects it; the regular build returns SOL_ATTN_ERR_UNSUPPORTED.  Copies up to
- * n (<= 32) counters, summed over CTAs, into cycles (host memory) after a device
+ * n (<= 48) counters, summed over CTAs, into cycles (host memory) after a device
  * synchronisation; reset != 0 clears them.  Slot order: the ProfSlot enum in
  * fused.cuh (wait cycles per role and barrier, per-role totals, softmax phases). */
 int sol_attn_profile_read(uint64_t* cycles, int n, int reset);
