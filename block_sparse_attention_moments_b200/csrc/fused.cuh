@@ -143,9 +143,10 @@ struct __align__(16) FusedCtl {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done[2];   // per softmax warpgroup (tile parity)
+  uint64_t s_full[3], p_full[3];    // per TMEM S buffer (tile index % 3)
+  uint64_t pv_done[3];              // per TMEM S buffer: its PV completed
   uint64_t xchg;                    // softmax warpgroups: partial row max / sum exchange
-  float xval[2][2][2][128];         // [phase parity][warpgroup][value][row]
+  float xval[2][2][128];            // [phase parity][warpgroup][row]
   uint32_t tmem_base;
   int abort;
 };
@@ -159,9 +160,9 @@ constexpr uint32_t kSmemV = kSmemK + kStages * kTile;
 constexpr uint32_t kSmemCtl = kSmemV + kStages * kTile;
 constexpr uint32_t kFusedSmemBytes = kSmemCtl + sizeof(FusedCtl) + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO0 = 0, kTmemS0 = 256;   // O_w at 128 w, S_w / P_w at 256 + 128 w
+constexpr uint32_t kTmemO = 0, kTmemS0 = 128;    // O at [0, 128), S / P buffer b at 128 + 128 b (b < 3)
 constexpr int kThreads = 384;
-constexpr int kSoftmaxThreads = 256;   // two warpgroups, each owning half of a tile's columns
+constexpr int kSoftmaxThreads = 256;   // two warpgroups, each owning half of every tile's columns
 constexpr uint32_t kRingEmptyCount = 8 + 3;  // softmax warps (lane 0 each) + K producer + V producer + MMA
 
 __device__ __forceinline__ bool mask_bit(const uint32_t* m, int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
@@ -290,6 +291,16 @@ struct TileIter {
 };
 
 
+// Bounded wait for an mbarrier phase after a failed first probe; on a timeout
+// it raises the abort flag and the status word.
+__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* status,
+                                       unsigned long long timeout_ns) {
+  if (mbar_wait(bar, parity, abort, timeout_ns)) return true;
+  *abort = 1;
+  atomicOr(status, kStatusTimeout);
+  return false;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     sol_attn_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -316,10 +327,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl.item_full[s], 1);
       mbar_init(&ctl.item_empty[s], 1);
-      mbar_init(&ctl.s_full[s], 1);
-      mbar_init(&ctl.p_full[s], kSoftmaxThreads / 2);
-      mbar_init(&ctl.o_done[s], 1);
     }
+    for (int b = 0; b < 3; ++b) {
+      mbar_init(&ctl.s_full[b], 1);
+      mbar_init(&ctl.p_full[b], kSoftmaxThreads);
+    }
+    for (int b = 0; b < 3; ++b) mbar_init(&ctl.pv_done[b], 1);
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&ctl.ring_full[r], 1);
       mbar_init(&ctl.ring_empty[r], kRingEmptyCount);
@@ -332,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ctl.q_full, 1);
     mbar_init(&ctl.q_empty, 1);
-    mbar_init(&ctl.xchg, kSoftmaxThreads);
+    mbar_init(&ctl.xchg, kSoftmaxThreads / 32);   // one arrival per softmax warp
     ctl.abort = 0;
     fence_mbar_init();
   }
@@ -350,15 +363,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // meets at the final barrier.
   SA_PROF(unsigned long long prof[kPrSlots]; for (int i = 0; i < kPrSlots; ++i) prof[i] = 0;
           const unsigned long long prof_t0 = clock64();)
+  // The first probe is inline; the sleeping loop behind it is out of line,
+  // which keeps every wait site small.
   auto wait = [&](uint64_t* bar, uint32_t parity, int slot) -> bool {
     SA_PROF(const unsigned long long tw = clock64();)
-    const bool okw = mbar_wait(bar, parity, abort_flag, p.timeout_ns);
+    const bool okw = mbar_try_wait(bar, parity) || wait_slow(bar, parity, abort_flag, p.status, p.timeout_ns);
     SA_PROF(prof[slot] += clock64() - tw;)
     (void)slot;
-    if (okw) return true;
-    *abort_flag = 1;
-    atomicOr(p.status, kStatusTimeout);
-    return false;
+    return okw;
   };
   // Consumer side of the descriptor ring: descriptor r lives in slot r % kRing.
   auto ring_get = [&](uint32_t r, int slot) -> bool {
@@ -578,38 +590,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // =========================================================== MMA issuer
+    // S(t) goes into TMEM buffer t % 3 and runs up to two tiles ahead of the
+    // PVs: for tile t this thread issues PV(t-2), then S(t) once PV(t-3), the
+    // last reader of the buffer, has completed.  PV(t-2) and S(t-1) sit
+    // between the two in the tensor pipe, so that wait rarely stalls it.
     if (lane == 0) {
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
+      const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
       int kstage = 0, vstage = 0;
       uint32_t kphase = 0, vphase = 0;
-      uint32_t tcount = 0;           // tiles whose S MMA is issued; tile t belongs to warpgroup t & 1
-      uint32_t wc0 = 0, wc1 = 0;     // tiles issued per warpgroup
+      uint32_t tcount = 0;           // tiles whose S MMA is issued
       uint32_t qseq = 0;             // items with tiles seen
-      bool seen0 = false, seen1 = false;   // warpgroup already had a tile in the current item
-      bool pend = false;             // the PV of the previous tile is still to be issued
-      int pv_ncols = 0, pv_w = 0, pv_stage = 0;
-      uint32_t pv_k = 0, pv_phase = 0;
-      bool pv_first = false;
+      struct PendingPv {
+        uint32_t t, vphase;
+        int ncols, vstage;
+        bool first;
+      };
+      PendingPv pend[2];
+      int npend = 0;
       bool ok = true;
-      // O_w (+)= P_w · Vside for the pending tile (P_w read from TMEM).
-      auto issue_pv = [&]() -> bool {
-        if (!wait(&ctl.p_full[pv_w], pv_k & 1, kPrMmaP)) return false;
-        if (!wait(&ctl.v_full[pv_stage], pv_phase, kPrMmaV)) return false;
+      // O (+)= P(t) · Vside(t), P read from TMEM buffer t % 3.  Softmax warpgroup
+      // w wrote the P of the tile's columns [w h, (w + 1) h), h = ncols / 2 (all
+      // 32 columns of a 32-column tile: warpgroup 0), as bf16 pairs starting at
+      // the buffer's column w h.
+      auto issue_pv = [&](const PendingPv& pv) -> bool {
+        const uint32_t b = pv.t % 3u;
+        if (!wait(&ctl.p_full[b], (pv.t / 3u) & 1u, kPrMmaP)) return false;
+        if (!wait(&ctl.v_full[pv.vstage], pv.vphase, kPrMmaV)) return false;
         tc_fence_after();
         SA_PROF(const unsigned long long tis = clock64();)
-        const int ksteps = pv_ncols / 16;
-        const uint32_t vbase = sVa + pv_stage * kTile;
-        const uint32_t pbase = tmem + kTmemS0 + 128 * pv_w;
-        const uint32_t dO = tmem + kTmemO0 + 128 * pv_w;
-        for (int kk = 0; kk < ksteps; ++kk)
-          umma_ts(dO, pbase + 8 * kk, sdesc_sw128(vbase + kk * 2048, CB, 1024), idesc_pv,
-                  (pv_first && kk == 0) ? 0u : 1u);
-        umma_commit(&ctl.o_done[pv_w]);
-        umma_commit(&ctl.v_empty[pv_stage]);
+        // descriptors are linear in the address: + (bytes >> 4) moves them
+        const uint64_t vdesc = sdesc_sw128(sVa + pv.vstage * kTile, CB, 1024);
+        const uint32_t pbase = tmem + kTmemS0 + 128u * b;
+        const uint32_t acc0 = pv.first ? 0u : 1u;
+        // K-step kk (keys 16 kk ..): P column 8 kk, + ncols / 4 for the second
+        // warpgroup's keys (a 32-column tile has only the first's)
+        if (pv.ncols == 128) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tmem + kTmemO, pbase + 8 * kk + (kk >= 4 ? 32 : 0), vdesc + 128 * kk, idesc_pv,
+                    kk == 0 ? acc0 : 1u);
+        } else if (pv.ncols == 64) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tmem + kTmemO, pbase + 8 * kk + (kk >= 2 ? 16 : 0), vdesc + 128 * kk, idesc_pv,
+                    kk == 0 ? acc0 : 1u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            umma_ts(tmem + kTmemO, pbase + 8 * kk, vdesc + 128 * kk, idesc_pv, kk == 0 ? acc0 : 1u);
+        }
+        umma_commit(&ctl.pv_done[b]);
+        umma_commit(&ctl.v_empty[pv.vstage]);
         SA_PROF(prof[kPrMmaIssuePV] += clock64() - tis;)
-        pend = false;
         return true;
+      };
+      auto pop_pv = [&]() -> bool {
+        const bool r = issue_pv(pend[0]);
+        pend[0] = pend[1];
+        --npend;
+        return r;
       };
       for (uint32_t r = 0;; ++r) {
         if (!ring_get(r, kPrMmaDesc)) { ok = false; break; }
@@ -618,36 +659,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&ctl.ring_empty[r % kRing]);
         if (flags & kDescEnd) break;
         if (flags & kDescEmpty) continue;
+        if (npend == 2 && !pop_pv()) { ok = false; break; }   // PV(t-2)
+        const uint32_t b = tcount % 3u;
+        if (tcount >= 3 && !wait(&ctl.pv_done[b], ((tcount / 3u) - 1u) & 1u, kPrMmaSEmpty)) { ok = false; break; }
         if (flags & kDescFirst) {
-          seen0 = seen1 = false;
           if (!wait(&ctl.q_full, qseq & 1, kPrMmaQ)) { ok = false; break; }
         }
-        const int w = tcount & 1;
-        const uint32_t k = w ? wc1 : wc0;
-        // S_w / P_w is free once the PV of this warpgroup's previous tile is done
-        if (k >= 1 && !wait(&ctl.o_done[w], (k - 1) & 1, kPrMmaSEmpty)) { ok = false; break; }
         if (!wait(&ctl.k_full[kstage], kphase, kPrMmaK)) { ok = false; break; }
         tc_fence_after();
         SA_PROF(const unsigned long long tis = clock64();)
-        // S(t) = Q · Kside^T into S_w
-        const uint32_t dS = tmem + kTmemS0 + 128 * w;
-        const uint32_t kbase = sKa + kstage * kTile;
+        // S(t) = Q · Kside^T into buffer t % 3
+        const uint32_t dS = tmem + kTmemS0 + 128u * b;
+        const uint64_t kdesc = sdesc_sw128(sKa + kstage * kTile, 16, 1024);
         const uint32_t idesc_s = idesc_bf16_f32(128, ncols, 0);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
-          const uint32_t koff = (kk >> 2) * CB + (kk & 3) * 32;
-          umma_ss(dS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(kbase + koff, 16, 1024), idesc_s,
-                  kk > 0 ? 1u : 0u);
+          const uint32_t koff = ((kk >> 2) * CB + (kk & 3) * 32) >> 4;
+          umma_ss(dS, qdesc + koff, kdesc + koff, idesc_s, kk > 0 ? 1u : 0u);
         }
         if (flags & kDescApprox) {  // + Q · K̄_lo^T (rows 64.. of the K-side tile)
 #pragma unroll
           for (int kk = 0; kk < KSTEPS; ++kk) {
-            const uint32_t koff = (kk >> 2) * CB + (kk & 3) * 32;
-            umma_ss(dS, sdesc_sw128(sQa + koff, 16, 1024), sdesc_sw128(kbase + 8192 + koff, 16, 1024),
-                    idesc_s, 1u);
+            const uint32_t koff = ((kk >> 2) * CB + (kk & 3) * 32) >> 4;
+            umma_ss(dS, qdesc + koff, kdesc + (8192 >> 4) + koff, idesc_s, 1u);
           }
         }
-        umma_commit(&ctl.s_full[w]);
+        umma_commit(&ctl.s_full[b]);
         umma_commit(&ctl.k_empty[kstage]);
         SA_PROF(prof[kPrMmaIssueS] += clock64() - tis;)
         if (++kstage == kStages) {
@@ -658,52 +695,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&ctl.q_empty);
           ++qseq;
         }
-        // PV of the previous tile, now that S(t) is queued ahead of it
-        if (pend && !issue_pv()) { ok = false; break; }
-        pend = true;
-        pv_ncols = ncols;
-        pv_w = w;
-        pv_k = k;
-        pv_first = w ? !seen1 : !seen0;
-        if (w) seen1 = true; else seen0 = true;
-        pv_stage = vstage;
-        pv_phase = vphase;
+        pend[npend++] = PendingPv{tcount, vphase, ncols, vstage, (flags & kDescFirst) != 0};
         if (++vstage == kStages) {
           vstage = 0;
           vphase ^= 1u;
         }
-        if (w) wc1 = k + 1; else wc0 = k + 1;
         ++tcount;
       }
-      if (ok && pend) issue_pv();
+      while (ok && npend > 0) ok = pop_pv();
     }
   } else {
     // =========================================================== softmax (warps 0-7)
-    // Warpgroup wg handles the tiles of parity wg, one thread per tile row
-    // and all of the row's columns; it keeps its own running max m, sum l and
-    // accumulator O_wg.  The two warpgroups meet once per item to merge.
+    // Both warpgroups work on every tile: the thread of warpgroup wg and TMEM
+    // lane `row` owns tile row `row` and the tile's columns [wg h, (wg + 1) h),
+    // h = ncols / 2 (a 32-column tile belongs to warpgroup 0 alone).  The two
+    // threads of a row share one reference maximum m (log2 units) and keep
+    // partial row sums l; P of the tile accumulates into the single O.
     const int wg = warp >> 2;
     const int row = tid & 127;        // tile row = TMEM lane
-    const int half = row >> 6;
+    const int half = row >> 6;        // query block of the pair the row belongs to
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + kTmemS0 + 128 * wg + lane_base;
-    const uint32_t tO_own = tmem + kTmemO0 + 128 * wg + lane_base;
-    uint32_t tcount = 0;     // tiles seen (both parities)
-    uint32_t kown = 0;       // own tiles processed
+    const uint32_t tO = tmem + kTmemO + lane_base;
+    uint32_t tcount = 0;     // tiles processed (S buffer tcount % 3, PV index tcount)
     uint32_t xc = 0;         // exchanges done
-    // Exchange two values per row with the other warpgroup.
-    auto exchange = [&](float a, float b2, float& oa, float& ob) {
+    // Exchange one value per row with the other warpgroup's thread of the row.
+    auto exchange = [&](float a) -> float {
       const int ph = xc & 1;
-      ctl.xval[ph][wg][0][row] = a;
-      ctl.xval[ph][wg][1][row] = b2;
-      mbar_arrive(&ctl.xchg);
+      ctl.xval[ph][wg][row] = a;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.xchg);
       wait(&ctl.xchg, ph, kPrSmX);
       ++xc;
-      oa = ctl.xval[ph][wg ^ 1][0][row];
-      ob = ctl.xval[ph][wg ^ 1][1][row];
+      return ctl.xval[ph][wg ^ 1][row];
     };
     float m_run = -INFINITY, l_run = 0.f;
-    bool own_any = false;    // this warpgroup had a tile in the current item
+    bool item_tiles = false;  // the current item had a tile
     for (uint32_t r = 0;; ++r) {
       if (!ring_get(r, kPrSmDesc)) break;
       const TileDesc& dsc = ctl.ring[r % kRing];
@@ -713,218 +739,181 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&ctl.ring_empty[r % kRing]);
       if (dflags & kDescEnd) break;
       if (!(dflags & kDescEmpty)) {
-        const bool mine = (tcount & 1) == static_cast<uint32_t>(wg);
-        ++tcount;
-        if (mine) {
-          wait(&ctl.s_full[wg], kown & 1, kPrSmS);
-          tc_fence_after();
-          SA_PROF(unsigned long long tph = clock64(); prof[kPrSmTiles] += 1;)
-          const int ng = ncols >> 5;   // 32-column groups: 1, 2 or 4
-          auto gb = [&](int i) -> uint32_t { return i == 0 ? bw.x : i == 1 ? bw.y : i == 2 ? bw.z : bw.w; };
-          // Column adjustments, only where needed: invalid columns become -inf,
-          // the ragged block's approximation column gets log2(n_tail / 64).
-          const int tail_g = tail_col >= 0 ? (tail_col >> 5) : -1;
-          auto adjust = [&](float* xv, int g) {
-            const uint32_t bits = gb(g);
-            const int et = (g == tail_g) ? (tail_col & 31) : -1;
-            if (bits != 0xFFFFFFFFu || et >= 0) {
+        const uint32_t t = tcount++;
+        const uint32_t b = t % 3u;
+        wait(&ctl.s_full[b], (t / 3u) & 1u, kPrSmS);
+        tc_fence_after();
+        SA_PROF(unsigned long long tph = clock64(); prof[kPrSmTiles] += 1;)
+        const bool first = (dflags & kDescFirst) != 0;
+        if (first) {
+          m_run = -INFINITY;
+          l_run = 0.f;
+        }
+        item_tiles = true;
+        const int hw = (ncols == 32) ? (wg == 0 ? 32 : 0) : (ncols >> 1);   // this thread's columns
+        const int c0 = (ncols == 32) ? 0 : wg * hw;                           // their first column
+        const int ng = hw >> 5;                                               // 32-column groups: 0, 1, 2
+        const uint32_t tS = tmem + kTmemS0 + 128u * b + lane_base;
+        auto gb = [&](int i) -> uint32_t { return i == 0 ? bw.x : i == 1 ? bw.y : i == 2 ? bw.z : bw.w; };
+        // Column adjustments, only where needed: invalid columns become -inf,
+        // the ragged block's approximation column gets log2(n_tail / 64).
+        const int tail_g = tail_col >= 0 ? (tail_col >> 5) : -1;
+        auto adjust = [&](float* xv, int g) {
+          const uint32_t bits = gb(g);
+          const int et = (g == tail_g) ? (tail_col & 31) : -1;
+          if (bits != 0xFFFFFFFFu || et >= 0) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                if (e == et) xv[e] += p.tail_raw;
-                if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
-              }
+            for (int e = 0; e < 32; ++e) {
+              if (e == et) xv[e] += p.tail_raw;
+              if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
             }
-          };
-          // In log2 units.  An approximation column stands for its n_j tokens:
-          // its weight n_j is folded into the logit as + log2(n_j) (6 for a full
-          // block) and the value side uses the block mean V̂_j / n_j.
-          const float boost = (dflags & kDescApprox) ? 6.f : 0.f;
-          const bool first_own = !own_any;
-          if (first_own) {
-            m_run = -INFINITY;
-            l_run = 0.f;
           }
-          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-          float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-          // p = 2^y, y = x * scale_log2 + off, for 32 adjusted columns, packed as
-          // 16 bf16 pairs; the fp32 values go into the row sum (ra, rb) and the
-          // largest y into ym.
-          auto probs32 = [&](const float* xv, float2 of2, uint32_t* pk, float2& ra, float2& rb, float& ym) {
+        };
+        // In log2 units.  An approximation column stands for its n_j tokens:
+        // its weight n_j is folded into the logit as + log2(n_j) (6 for a full
+        // block) and the value side uses the block mean V̂_j / n_j.
+        const float boost = (dflags & kDescApprox) ? 6.f : 0.f;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        // p = 2^y, y = x * scale_log2 + off, for 32 adjusted columns, packed as
+        // 16 bf16 pairs; the fp32 values go into the row sum (ra, rb) and the
+        // largest y into ym.
+        auto probs32 = [&](const float* xv, float2 of2, uint32_t* pk, float2& ra, float2& rb, float& ym) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
-              const float2 y1 = __ffma2_rn(make_float2(xv[e + 2], xv[e + 3]), sc2, of2);
-              const float2 y2 = __ffma2_rn(make_float2(xv[e + 4], xv[e + 5]), sc2, of2);
-              const float2 y3 = __ffma2_rn(make_float2(xv[e + 6], xv[e + 7]), sc2, of2);
-              ym = max3f(ym, max3f(y0.x, y0.y, y1.x), max3f(y1.y, y2.x, y2.y));
-              ym = max3f(ym, y3.x, y3.y);
-              const float2 q0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
-              const float2 q1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
-              const float2 q2 = make_float2(ex2_approx(y2.x), ex2_approx(y2.y));
-              const float2 q3 = make_float2(ex2_approx(y3.x), ex2_approx(y3.y));
-              ra = __fadd2_rn(ra, __fadd2_rn(q0, q2));
-              rb = __fadd2_rn(rb, __fadd2_rn(q1, q3));
-              pk[e >> 1] = pack_bf16x2(q0.x, q0.y);
-              pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
-              pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
-              pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
-            }
-          };
-          // Read, adjust and exponentiate groups g0 and g0 + 1 (those below ng)
-          // into pk[0, 32); returns the largest y.
-          auto half_tile = [&](int g0, float2 of2, uint32_t* pk, float2& ra, float2& rb) -> float {
-            float ym = -INFINITY;
+          for (int e = 0; e < 32; e += 8) {
+            const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
+            const float2 y1 = __ffma2_rn(make_float2(xv[e + 2], xv[e + 3]), sc2, of2);
+            const float2 y2 = __ffma2_rn(make_float2(xv[e + 4], xv[e + 5]), sc2, of2);
+            const float2 y3 = __ffma2_rn(make_float2(xv[e + 6], xv[e + 7]), sc2, of2);
+            ym = max3f(ym, max3f(y0.x, y0.y, y1.x), max3f(y1.y, y2.x, y2.y));
+            ym = max3f(ym, y3.x, y3.y);
+            const float2 q0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+            const float2 q1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+            const float2 q2 = make_float2(ex2_approx(y2.x), ex2_approx(y2.y));
+            const float2 q3 = make_float2(ex2_approx(y3.x), ex2_approx(y3.y));
+            ra = __fadd2_rn(ra, __fadd2_rn(q0, q2));
+            rb = __fadd2_rn(rb, __fadd2_rn(q1, q3));
+            pk[e >> 1] = pack_bf16x2(q0.x, q0.y);
+            pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
+            pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
+            pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
+          }
+        };
+        // This thread's columns, against the reference maximum mref: P into
+        // pk[0, 16 ng), the row sum into (ra, rb); returns the largest y.
+        auto own_cols = [&](float mref, uint32_t* pk, float2& ra, float2& rb) -> float {
+          const float2 of2 = make_float2(boost - mref, boost - mref);
+          float ym = -INFINITY;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (g0 + h < ng) {
-                float xv[32];
-                tmem_ld_x32f(tS + 32 * (g0 + h), xv);
-                tmem_ld_wait();
-                reg_fence32(xv);
-                adjust(xv, g0 + h);
-                probs32(xv, of2, pk + 16 * h, ra, rb, ym);
-              }
+          for (int i = 0; i < 2; ++i) {
+            if (i < ng) {
+              float xv[32];
+              tmem_ld_x32f(tS + c0 + 32 * i, xv);
+              tmem_ld_wait();
+              reg_fence32(xv);
+              adjust(xv, (c0 >> 5) + i);
+              probs32(xv, of2, pk + 16 * i, ra, rb, ym);
             }
-            return ym;
-          };
-          // O_wg *= alpha (per row).  O_wg holds this warpgroup's previous tiles;
-          // their PVs completed before the MMA issuer wrote this S tile (it waits
-          // for them), so O_wg is stable.
-          auto rescale_o = [&](float alpha) {
-            SA_PROF(prof[kPrSmRescales] += 1;)
+          }
+          return ym;
+        };
+        // One pass against the row's reference maximum m (0 while the row has
+        // seen no valid column), P held in registers.  Each thread proposes the
+        // m it needs: m itself while its y stay <= 8 (the lazy rescale rule),
+        // else m raised by a whole number k of doublings (so that everything
+        // accumulated so far scales by 2^-k exactly, even P already in bf16),
+        // or its maximum rounded up on the row's first valid column.  The two
+        // threads of the row agree on the larger proposal; where it moved, l
+        // and this thread's half of O scale by 2^(m - m') and the columns are
+        // recomputed from S, which no P store has reached yet.
+        uint32_t pk[32];
+        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+        const float ym = own_cols(m_run == -INFINITY ? 0.f : m_run, pk, sa, sb);
+        // m stays a whole number (its first value is rounded up), so that every
+        // later step m' - m is exact in fp32
+        const float prop = (m_run == -INFINITY) ? ceilf(ym) : (ym > 8.f ? m_run + ceilf(ym) : m_run);
+        const float m_new = fmaxf(prop, exchange(prop));
+        const bool moved = !(m_new == m_run);
+        if (__any_sync(0xFFFFFFFFu, moved)) {
+          SA_PROF(prof[kPrSmRedo] += 1;)
+          float alpha = 1.f;
+          if (moved) {
+            if (m_run == -INFINITY) {
+              alpha = 0.f;   // nothing valid accumulated yet
+            } else {
+              const int k = __float2int_rn(m_new - m_run);
+              alpha = (k >= 126) ? 0.f : __int_as_float((127 - k) << 23);
+            }
+            l_run *= alpha;
+            m_run = m_new;
+          }
+          __syncwarp();
+          if (!first) {
+            // O holds PV(0 .. t-1) of the item; wait for PV(t-1), then scale this
+            // thread's half of the row
+            wait(&ctl.pv_done[(t - 1u) % 3u], ((t - 1u) / 3u) & 1u, kPrSmO);
+            tc_fence_after();
 #pragma unroll 1
-            for (int c16 = 0; c16 < D; c16 += 16) {
+            for (int c16 = wg * (D / 2); c16 < (wg + 1) * (D / 2); c16 += 16) {
               float rr[16];
-              tmem_ld_x16f(tO_own + c16, rr);
+              tmem_ld_x16f(tO + c16, rr);
               tmem_ld_wait();
               reg_fence16(rr);
               uint32_t pw[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) pw[e] = __float_as_uint(rr[e] * alpha);
-              tmem_st_x16(tO_own + c16, pw);
+              tmem_st_x16(tO + c16, pw);
             }
-          };
-          // One pass over S, 64 columns (a half) at a time, against the current
-          // reference maximum m (0 while the row has seen no valid column).  P
-          // of a half stays in registers until the half's largest y is known:
-          // while every row of the warp has y <= 8 the lazy rescale rule keeps m
-          // and P lands in TMEM as computed.  Otherwise the rows past the limit
-          // raise m (to their maximum on a first valid column, else by a whole
-          // number k of doublings, so that the values already accumulated scale
-          // by 2^-k exactly, even P already in bf16) and the half is recomputed
-          // from S, which no P store has reached yet: half h's P goes to
-          // columns [32h, 32h + 32), over S groups that were read before it.
-          const int nh = (ng + 1) >> 1;
-          int redo = 0;   // recomputations of the current half (one suffices; two bound the loop)
-#pragma unroll 1
-          for (int h = 0; h < nh;) {
-            const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-            const float2 of2 = make_float2(boost - mref, boost - mref);
-            float2 ha = make_float2(0.f, 0.f), hb = make_float2(0.f, 0.f);
-            uint32_t pk[32];
-            const float ym = half_tile(2 * h, of2, pk, ha, hb);
-            const bool ex = (m_run == -INFINITY) ? (ym != -INFINITY) : (ym > 8.f);
-            if (redo < 2 && __any_sync(0xFFFFFFFFu, ex)) {
-              ++redo;
-              SA_PROF(prof[kPrSmRedo] += 1;)
-              float alpha = 1.f;
-              if (ex) {
-                if (m_run == -INFINITY) {
-                  m_run = ym;       // y was measured against 0: this is the maximum itself
-                  alpha = 0.f;      // nothing valid accumulated yet
-                } else {
-                  const float k = ceilf(ym);
-                  m_run += k;
-                  alpha = (k >= 126.f) ? 0.f : __int_as_float((127 - static_cast<int>(k)) << 23);
-                }
-                l_run *= alpha;
-                sa = make_float2(sa.x * alpha, sa.y * alpha);
-                sb = make_float2(sb.x * alpha, sb.y * alpha);
-              }
-              __syncwarp();
-              if (h > 0) {   // P of columns [0, 64), already in TMEM columns [0, 32)
-                tmem_st_wait();
-#pragma unroll 1
-                for (int c16 = 0; c16 < 32; c16 += 16) {
-                  float rr[16];
-                  tmem_ld_x16f(tS + c16, rr);
-                  tmem_ld_wait();
-                  reg_fence16(rr);
-                  uint32_t pw[16];
-#pragma unroll
-                  for (int e = 0; e < 16; ++e) {
-                    const uint32_t u = __float_as_uint(rr[e]);
-                    pw[e] = pack_bf16x2(__uint_as_float(u << 16) * alpha, __uint_as_float(u & 0xFFFF0000u) * alpha);
-                  }
-                  tmem_st_x16(tS + c16, pw);
-                }
-              }
-              if (!first_own) rescale_o(alpha);
-              continue;   // the same half again, against the new m
-            }
-            tmem_st_x16(tS + 32 * h, pk);
-            if (2 * h + 1 < ng) tmem_st_x16(tS + 32 * h + 16, pk + 16);
-            sa = __fadd2_rn(sa, ha);
-            sb = __fadd2_rn(sb, hb);
-            ++h;
-            redo = 0;
+            SA_PROF(prof[kPrSmRescales] += 1;)
           }
-          l_run += (sa.x + sa.y) + (sb.x + sb.y);
-          tmem_st_wait();
-          SA_PROF(prof[kPrSmPass2] += clock64() - tph;)
-          tc_fence_before();
-          mbar_arrive(&ctl.p_full[wg]);
-          ++kown;
-          own_any = true;
+          sa = make_float2(0.f, 0.f);
+          sb = make_float2(0.f, 0.f);
+          (void)own_cols(m_run == -INFINITY ? 0.f : m_run, pk, sa, sb);
         }
+        // P of this thread's columns lands in TMEM columns [c0, c0 + hw / 2),
+        // inside its own part of S, which it has read
+        if (ng > 0) tmem_st_x16(tS + c0, pk);
+        if (ng > 1) tmem_st_x16(tS + c0 + 16, pk + 16);
+        l_run += (sa.x + sa.y) + (sb.x + sb.y);
+        tmem_st_wait();
+        SA_PROF(prof[kPrSmPass2] += clock64() - tph;)
+        tc_fence_before();
+        mbar_arrive(&ctl.p_full[b]);
       }
       if (!(dflags & (kDescLast | kDescEmpty))) continue;
-      // ---- epilogue: merge the two warpgroups' partial softmaxes (Eq. 10)
+      // ---- epilogue: O / (l_0 + l_1) for this thread's half of the row's columns
       SA_PROF(const unsigned long long tep = clock64();)
-      if (own_any) {   // this warpgroup's last PV
-        wait(&ctl.o_done[wg], (kown - 1) & 1, kPrSmO);
+      if (item_tiles) {   // the item's last PV
+        wait(&ctl.pv_done[(tcount - 1u) % 3u], ((tcount - 1u) / 3u) & 1u, kPrSmO);
         tc_fence_after();
       }
-      const float my_m = own_any ? m_run : -INFINITY;
-      const float my_l = own_any ? l_run : 0.f;
-      float ot_m, ot_l;
-      exchange(my_m, my_l, ot_m, ot_l);
-      tc_fence_after();
-      const float mm = fmaxf(my_m, ot_m);
-      const float f_own = (my_m == -INFINITY) ? 0.f : ex2_approx(my_m - mm);
-      const float f_oth = (ot_m == -INFINITY) ? 0.f : ex2_approx(ot_m - mm);
-      const float l_tot = f_own * my_l + f_oth * ot_l;
+      const float my_l = item_tiles ? l_run : 0.f;
+      const float l_tot = my_l + exchange(my_l);
       const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
-      const float w_own = f_own * inv_l, w_oth = f_oth * inv_l;
-      const bool own_has = own_any && w_own != 0.f, oth_has = (ot_m != -INFINITY) && w_oth != 0.f;
       const int token = 128 * dpair + row;
       uint16_t* orow = p.out + (static_cast<size_t>(dbh) * p.L + token) * D;
-      // warpgroup wg writes O columns [wg * D/2, (wg + 1) * D/2), 16 at a time
 #pragma unroll 1
-      for (int c16 = wg * D / 32; c16 < (wg + 1) * D / 32; ++c16) {
-        float a[16], c[16];
-        if (own_has) tmem_ld_x16f(tmem + kTmemO0 + 128 * wg + lane_base + c16 * 16, a);
-        if (oth_has) tmem_ld_x16f(tmem + kTmemO0 + 128 * (wg ^ 1) + lane_base + c16 * 16, c);
-        tmem_ld_wait();
-        reg_fence16(a);
-        reg_fence16(c);
-        if (token < p.L) {
+      for (int c16 = wg * (D / 2); c16 < (wg + 1) * (D / 2); c16 += 16) {
+        float a[16];
+        if (item_tiles) {
+          tmem_ld_x16f(tO + c16, a);
+          tmem_ld_wait();
+          reg_fence16(a);
+        } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            a[e] = (own_has ? a[e] * w_own : 0.f) + (oth_has ? c[e] * w_oth : 0.f);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c16 * 16);
-          dst[0] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
-                              pack_bf16x2(a[6], a[7]));
-          dst[1] = make_uint4(pack_bf16x2(a[8], a[9]), pack_bf16x2(a[10], a[11]), pack_bf16x2(a[12], a[13]),
-                              pack_bf16x2(a[14], a[15]));
+          for (int e = 0; e < 16; ++e) a[e] = 0.f;
+        }
+        if (token < p.L) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c16);
+          dst[0] = make_uint4(pack_bf16x2(a[0] * inv_l, a[1] * inv_l), pack_bf16x2(a[2] * inv_l, a[3] * inv_l),
+                              pack_bf16x2(a[4] * inv_l, a[5] * inv_l), pack_bf16x2(a[6] * inv_l, a[7] * inv_l));
+          dst[1] = make_uint4(pack_bf16x2(a[8] * inv_l, a[9] * inv_l), pack_bf16x2(a[10] * inv_l, a[11] * inv_l),
+                              pack_bf16x2(a[12] * inv_l, a[13] * inv_l), pack_bf16x2(a[14] * inv_l, a[15] * inv_l));
         }
       }
-      // both warpgroups are done reading O_0 and O_1 before either can start
-      // the next item (whose first PVs overwrite them)
+      // O is read; the next item's first PV (which overwrites O) waits for this
+      // thread's next P arrival, which comes after these reads
       tc_fence_before();
-      float d0, d1;
-      exchange(0.f, 0.f, d0, d1);
-      own_any = false;
+      item_tiles = false;
       SA_PROF(prof[kPrSmEpi] += clock64() - tep;)
     }
   }
