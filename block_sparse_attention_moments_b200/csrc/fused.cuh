@@ -15,24 +15,26 @@
 // blocks reach that half through the approximation instead).  The result is
 // the same as processing the blocks one by one.
 //
-// For each chunk t of C pooled keys (outer loop) the item's tile sequence is
-//   approx  A = Q·K̄^(t)ᵀ (128 x W, W = 32 or 64 pooled keys; K̄ as a bf16 hi/lo
-//           pair so the logits keep K̄ to ~16 bits); per row, columns not
-//           selected by the row's half get p = n_j 2^(a-m) (n_j folded into the
-//           logit as + log2 n_j), l += p and O += p V̄_j with V̄_j = V̂_j / n_j,
-//           which is Eq. 9-10's n_j e^a in the denominator and e^a V̂_j above;
+// For each chunk of C pooled keys the item's tile sequence holds
 //   exact   the selected blocks of the chunk, two per tile: S = Q·[K_a;K_b]ᵀ
 //           (128 x 128), per-half / key >= L masks, online-softmax update,
-//           O += P·[V_a;V_b].
-// Epilogue: O / l in bf16 for rows < L.
+//           O += P·[V_a;V_b];
+//   approx  A = Q·K̄ᵀ over the chunk's pooled keys (128 x W, W = 32 or 64; K̄
+//           as a bf16 hi/lo pair so the logits keep K̄ to ~16 bits); per row,
+//           columns not selected by the row's half get p = n_j 2^(a-m) (n_j
+//           folded into the logit as + log2 n_j), l += p and O += p V̄_j with
+//           V̄_j = V̂_j / n_j, which is Eq. 9-10's n_j e^a in the denominator
+//           and e^a V̂_j above.
+// The walk starts at the chunk holding the item's own query blocks (see
+// TileIter).  Epilogue: O / l in bf16 for rows < L.
 //
 // Warp roles (384 threads, one persistent CTA per SM, atomic work counter):
 //   warps 0-7  softmax, two warpgroups: each thread owns one tile row and one
-//              half of the tile's columns; masks, lazy-rescaled online
-//              softmax, P to shared memory, O correction in TMEM, epilogue.
+//              half of every tile's columns; masks, lazy-rescaled one-pass
+//              online softmax, P into TMEM, epilogue.
 //   warp 8     TMA producers: lane 0 loads Q and the K side (K blocks, or K̄
 //              hi/lo), lane 1 the V side (V blocks, or V̄).
-//   warp 9     tcgen05 MMA issuer: S(t+1) is issued before PV(t).
+//   warp 9     tcgen05 MMA issuer: S runs up to two tiles ahead of the PVs.
 //   warp 10    routing: fetches the next item, computes ŝ_ij = Q̄_i·K̄_j/sqrt(d)
 //              in fp32 for both halves, compares with τ_i (warp ballot -> mask
 //              words), one item ahead (double-buffered mask slots).
@@ -41,17 +43,15 @@
 //              half, first/last flags) into a shared-memory ring that the
 //              producers, the MMA issuer and the softmax warps consume.
 //
-// Tiles alternate between the two softmax warpgroups (global tile index
-// parity w): warpgroup w owns every row of its tiles, keeps its own running
-// max / sum, and accumulates into its own O_w.  At the end of an item the two
-// partial results are merged, O = (2^(m0-m) O_0 + 2^(m1-m) O_1) / (2^(m0-m) l_0
-// + 2^(m1-m) l_1), the usual combination of partial online softmaxes.  P is
-// written back into TMEM over its S tile (bf16 pairs) and fed to the PV MMA
-// as its A operand, so the only shared-memory operand traffic is Q, K and V.
+// The two threads of a row (one per warpgroup) share one reference maximum,
+// agreed per tile through shared memory, so a single O accumulates the whole
+// row.  P is written back into TMEM over the thread's own part of its S tile
+// (bf16 pairs) and fed to the PV MMA as its A operand, so the only
+// shared-memory operand traffic is Q, K and V.
 //
 // Shared memory (1024-byte aligned, 128-byte swizzled tiles):
 //   Q 32 KB | K ring 2 x 32 KB | V ring 2 x 32 KB | control.
-// TMEM (512 columns): O_0 [0,128), O_1 [128,256), S_0/P_0 [256,384), S_1/P_1 [384,512).
+// TMEM (512 columns): O [0,128), S/P buffers b = t mod 3 at [128 + 128 b, 256 + 128 b).
 #pragma once
 
 #include <cstddef>
