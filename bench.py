@@ -254,6 +254,42 @@ def run_role_profile(args):
                                                        "softmax.wait_exchange")}}), flush=True)
 
 
+def run_ablation(args):
+    """Approximation ablation (not a bench line): for each beta, the output of the
+    full method and of the exact-only variant (no approximation of unselected
+    blocks, same selection) against the select-all output of the same kernel,
+    as relative l2 error and mean per-row cosine similarity.  "Sol-Attn: ...",
+    experiments: ablation of the proxy-score approximation."""
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_moments_b200 as sa
+    from synth import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    qb, kb, vb = rank_inputs(wl, 0)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = dev(qb), dev(kb), dev(vb)
+    dense = sa.forward(q, k, v, -math.inf, wl.chunk, flags=sa.FLAG_SELECT_ALL).float()
+
+    def compare(o):
+        o = o.float()
+        rel = (torch.linalg.vector_norm(o - dense) / torch.linalg.vector_norm(dense)).item()
+        cos = torch.nn.functional.cosine_similarity(o.reshape(-1, o.shape[-1]), dense.reshape(-1, o.shape[-1]),
+                                                    dim=-1).mean().item()
+        return rel, cos
+
+    for beta in args.ablation_betas:
+        o_full = sa.forward(q, k, v, beta, wl.chunk)
+        counts = sa.stats(wl.B, wl.H, wl.L)
+        density = counts.double().mean().item() / counts.shape[-1]
+        o_exact = sa.forward(q, k, v, beta, wl.chunk, flags=sa.FLAG_EXACT_ONLY)
+        rf, cf = compare(o_full)
+        re, ce = compare(o_exact)
+        print(json.dumps({"mode": "ablation", "workload": wl.name, "beta": beta, "density": density,
+                          "approx": {"rel_l2_vs_dense": rf, "cosine_vs_dense": cf},
+                          "exact_only": {"rel_l2_vs_dense": re, "cosine_vs_dense": ce}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -267,11 +303,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the select-all (dense) comparison run")
+    ap.add_argument("--ablation", action="store_true",
+                    help="approximation ablation: full method and exact-only against select-all (not a bench line)")
+    ap.add_argument("--ablation-betas", type=float, nargs="+", default=[0.75, 1.0, 1.5])
     ap.add_argument("--role-profile", action="store_true",
                     help="run the profiling build (libsol_attn_profile.so) and print per-role cycle accounting")
     args = ap.parse_args()
     if args.role_profile:
         return run_role_profile(args)
+    if args.ablation:
+        return run_ablation(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

@@ -163,3 +163,22 @@ def test_runtime_errors_on_device():
     with pytest.raises(sa.SolAttnError) as e:
         sa.stage_fused(q, k, v, torch.empty_like(q), 4) if False else sa.stage_threshold(1, 3, 1024, 64, 1.0)
     assert e.value.code == -6
+
+
+@pytest.mark.parametrize("beta", [0.75, 1.0, 1.5])
+def test_approximation_ablation_on_device(beta):
+    # experiments, ablation of the proxy-score approximation: on the same
+    # selection, adding the approximation of the unselected blocks brings the
+    # output closer to full attention than dropping them (exact-only)
+    import torch
+    wl = WORKLOADS["image"]
+    qb, kb, vb = fourier_inputs(wl)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = dev(qb), dev(kb), dev(vb)
+    dense = sa.forward(q, k, v, -math.inf, wl.chunk, flags=sa.FLAG_SELECT_ALL).float()
+    full = sa.forward(q, k, v, beta, wl.chunk).float()
+    exact = sa.forward(q, k, v, beta, wl.chunk, flags=sa.FLAG_EXACT_ONLY).float()
+    rel = lambda o: (torch.linalg.vector_norm(o - dense) / torch.linalg.vector_norm(dense)).item()
+    r_full, r_exact = rel(full), rel(exact)
+    print(f"beta={beta} rel-l2 vs select-all: approx {r_full:.4f} exact-only {r_exact:.4f}")
+    assert 0.0 < r_full < r_exact
