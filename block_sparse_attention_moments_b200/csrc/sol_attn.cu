@@ -68,10 +68,14 @@ struct Workspace {
   Shape shape;        // shape the views are carved for
   int stage = 0;      // 0 none, 1 pooled, 2 thresholds, 3 fused done
   Shape last_fused;   // shape of the last completed forward (for stats)
-  // host-buffer entry point staging
+  // host-buffer entry point: two staging slots, three streams (copy in,
+  // compute, copy out) and the events that order them
   void* host_stage = nullptr;
   size_t host_stage_bytes = 0;
-  cudaStream_t host_stream = nullptr;
+  cudaStream_t host_stream = nullptr;   // copies in
+  cudaStream_t host_comp = nullptr;     // kernels
+  cudaStream_t host_out = nullptr;      // copies out
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
 };
 
 constexpr int kMaxDevices = 64;
@@ -491,37 +495,73 @@ int sol_attn_forward_host(const uint16_t* q, const uint16_t* k, const uint16_t* 
   int rc;
   if ((rc = check_shape(B, H, L, d, block))) return rc;
   if (!q || !k || !v || !out) return fail(SOL_ATTN_ERR_ARG, "a host pointer is NULL");
+  if (chunk < 1) return fail(SOL_ATTN_ERR_ARG, "chunk must be >= 1 (got %d)", chunk);
+  if (std::isnan(beta)) return fail(SOL_ATTN_ERR_ARG, "beta is NaN");
   int dev;
   if ((rc = current_device(&dev))) return rc;
-  const size_t n = static_cast<size_t>(B) * H * L * d * 2;
-  const size_t per = align_up(n, 256);
-  char* dq;
-  cudaStream_t st;
+  // The (batch, head) slices are independent and contiguous: they go through in
+  // up to kHostChunks groups, the copy in of group c + 1 and the copy out of
+  // group c - 1 overlapping the kernels of group c.
+  constexpr int kHostChunks = 8;
+  const int BH = B * H;
+  const int hc = (BH + kHostChunks - 1) / kHostChunks;     // heads per group
+  const int ngroups = (BH + hc - 1) / hc;
+  const size_t head_elems = static_cast<size_t>(L) * d;
+  const size_t slot = align_up(static_cast<size_t>(hc) * head_elems * 2, 256);   // one tensor of a group
+  Workspace* w;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    Workspace& w = g_ws[dev];
-    if (!w.host_stream) CUDA_TRY(cudaStreamCreateWithFlags(&w.host_stream, cudaStreamNonBlocking));
-    if (w.host_stage_bytes < 4 * per) {
-      if (w.host_stage) CUDA_TRY(cudaFree(w.host_stage));
-      w.host_stage = nullptr;
-      w.host_stage_bytes = 0;
-      CUDA_TRY(cudaMalloc(&w.host_stage, 4 * per));
-      w.host_stage_bytes = 4 * per;
+    w = &g_ws[dev];
+    if (!w->host_stream) {
+      CUDA_TRY(cudaStreamCreateWithFlags(&w->host_stream, cudaStreamNonBlocking));
+      CUDA_TRY(cudaStreamCreateWithFlags(&w->host_comp, cudaStreamNonBlocking));
+      CUDA_TRY(cudaStreamCreateWithFlags(&w->host_out, cudaStreamNonBlocking));
+      for (int i = 0; i < 2; ++i) {
+        CUDA_TRY(cudaEventCreateWithFlags(&w->ev_in[i], cudaEventDisableTiming));
+        CUDA_TRY(cudaEventCreateWithFlags(&w->ev_comp[i], cudaEventDisableTiming));
+        CUDA_TRY(cudaEventCreateWithFlags(&w->ev_out[i], cudaEventDisableTiming));
+      }
     }
-    dq = static_cast<char*>(w.host_stage);
-    st = w.host_stream;
+    if (w->host_stage_bytes < 8 * slot) {   // 2 slots x (q, k, v, out)
+      if (w->host_stage) CUDA_TRY(cudaFree(w->host_stage));
+      w->host_stage = nullptr;
+      w->host_stage_bytes = 0;
+      CUDA_TRY(cudaMalloc(&w->host_stage, 8 * slot));
+      w->host_stage_bytes = 8 * slot;
+    }
   }
-  CUDA_TRY(cudaMemcpyAsync(dq, q, n, cudaMemcpyHostToDevice, st));
-  CUDA_TRY(cudaMemcpyAsync(dq + per, k, n, cudaMemcpyHostToDevice, st));
-  CUDA_TRY(cudaMemcpyAsync(dq + 2 * per, v, n, cudaMemcpyHostToDevice, st));
-  rc = sol_attn_forward_ex(dq, dq + per, dq + 2 * per, dq + 3 * per, B, H, L, d, block, chunk, beta,
-                           flags & ~SOL_ATTN_FLAG_SYNC_CHECK, nullptr, st);
-  if (rc) return rc;
-  CUDA_TRY(cudaMemcpyAsync(out, dq + 3 * per, n, cudaMemcpyDeviceToHost, st));
-  CUDA_TRY(cudaStreamSynchronize(st));
+  char* stage = static_cast<char*>(w->host_stage);
+  cudaStream_t s_in = w->host_stream, s_comp = w->host_comp, s_out = w->host_out;
+  for (int c = 0; c < ngroups; ++c) {
+    const int sl = c & 1;
+    const int h0 = c * hc, cnt = std::min(hc, BH - h0);
+    const size_t off = static_cast<size_t>(h0) * head_elems, bytes = static_cast<size_t>(cnt) * head_elems * 2;
+    char* dq = stage + (4 * sl) * slot;
+    char* dk = dq + slot;
+    char* dv = dq + 2 * slot;
+    char* dout = dq + 3 * slot;
+    // inputs of slot sl are free once the kernels of group c - 2 have run
+    if (c >= 2) CUDA_TRY(cudaStreamWaitEvent(s_in, w->ev_comp[sl], 0));
+    CUDA_TRY(cudaMemcpyAsync(dq, q + off, bytes, cudaMemcpyHostToDevice, s_in));
+    CUDA_TRY(cudaMemcpyAsync(dk, k + off, bytes, cudaMemcpyHostToDevice, s_in));
+    CUDA_TRY(cudaMemcpyAsync(dv, v + off, bytes, cudaMemcpyHostToDevice, s_in));
+    CUDA_TRY(cudaEventRecord(w->ev_in[sl], s_in));
+    CUDA_TRY(cudaStreamWaitEvent(s_comp, w->ev_in[sl], 0));
+    // the output of slot sl is free once group c - 2 has been copied out
+    if (c >= 2) CUDA_TRY(cudaStreamWaitEvent(s_comp, w->ev_out[sl], 0));
+    rc = sol_attn_forward_ex(dq, dk, dv, dout, 1, cnt, L, d, block, chunk, beta, flags & ~SOL_ATTN_FLAG_SYNC_CHECK,
+                             nullptr, s_comp);
+    if (rc) return rc;
+    CUDA_TRY(cudaEventRecord(w->ev_comp[sl], s_comp));
+    CUDA_TRY(cudaStreamWaitEvent(s_out, w->ev_comp[sl], 0));
+    CUDA_TRY(cudaMemcpyAsync(out + off, dout, bytes, cudaMemcpyDeviceToHost, s_out));
+    CUDA_TRY(cudaEventRecord(w->ev_out[sl], s_out));
+  }
+  CUDA_TRY(cudaStreamSynchronize(s_out));
+  CUDA_TRY(cudaStreamSynchronize(s_comp));
   if (flags & SOL_ATTN_FLAG_SYNC_CHECK) {
     std::lock_guard<std::mutex> lk(g_mu);
-    return read_status(g_ws[dev], st);
+    return read_status(g_ws[dev], s_comp);
   }
   return SOL_ATTN_OK;
 }
@@ -540,6 +580,13 @@ int sol_attn_release(void) {
   if (w.ctl_block) CUDA_TRY(cudaFree(w.ctl_block));
   if (w.host_stage) CUDA_TRY(cudaFree(w.host_stage));
   if (w.host_stream) CUDA_TRY(cudaStreamDestroy(w.host_stream));
+  if (w.host_comp) CUDA_TRY(cudaStreamDestroy(w.host_comp));
+  if (w.host_out) CUDA_TRY(cudaStreamDestroy(w.host_out));
+  for (int i = 0; i < 2; ++i) {
+    if (w.ev_in[i]) CUDA_TRY(cudaEventDestroy(w.ev_in[i]));
+    if (w.ev_comp[i]) CUDA_TRY(cudaEventDestroy(w.ev_comp[i]));
+    if (w.ev_out[i]) CUDA_TRY(cudaEventDestroy(w.ev_out[i]));
+  }
   w = Workspace{};
   return SOL_ATTN_OK;
 }

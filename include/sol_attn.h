@@ -97,9 +97,13 @@ int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out,
  * if the last forward had a different (B,H,L,block). */
 int sol_attn_stats(int32_t* counts, int B, int H, int L, int block, void* stream);
 
-/* End-to-end call on HOST buffers (pinned or pageable): copies q, k, v to the
- * device, runs sol_attn_forward_ex on an internal stream, copies out back and
- * synchronises.  Device staging buffers are owned and cached by the library. */
+/* End-to-end call on HOST buffers (pinned or pageable; pinned lets the copies
+ * overlap): the B*H independent (batch, head) slices go through in up to 8
+ * groups; for each group q, k, v are copied to the device, sol_attn_forward_ex
+ * runs on the group and out is copied back, on three internal streams so that
+ * the copies of neighbouring groups overlap the kernels.  Synchronises before
+ * returning.  Device staging buffers (two groups) are owned and cached by the
+ * library.  sol_attn_stats afterwards refers to the last group only. */
 int sol_attn_forward_host(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                           uint16_t* out, int B, int H, int L, int d, int block,
                           int chunk, float beta, unsigned flags);

@@ -130,6 +130,17 @@ def test_host_buffer_entry_point_matches_device_call():
     assert np.array_equal(got, dev)
 
 
+def test_host_buffer_entry_point_in_groups():
+    # 9 (batch, head) slices go through in 5 groups of 2, 2, 2, 2 and 1: the
+    # result equals one device call on all of them, bit for bit
+    import torch
+    qb, kb, vb = gauss_inputs(3, 3, 1000, 64, seed=77)
+    dev, _, _ = run_gpu(qb, kb, vb, 0.75, 5, debug=False)
+    host = sa.forward_host(qb, kb, vb, 0.75, 5, flags=sa.FLAG_SYNC_CHECK)
+    got = torch.from_numpy(host.view(np.int16)).view(torch.bfloat16).float().numpy()
+    assert np.array_equal(got, dev)
+
+
 def test_staged_calls_match_forward():
     import torch
     from parity_util import to_device
