@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j < p.N) {
           const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
-#pragma unroll 8
+#pragma unroll 2
           for (int c4 = 0; c4 < D / 4; ++c4) {
             const float4 x = __ldg(kr + c4);
             const float4 qa = *reinterpret_cast<const float4*>(&ctl.qbar[0][4 * c4]);
