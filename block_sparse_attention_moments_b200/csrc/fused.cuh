@@ -141,8 +141,8 @@ struct __align__(16) FusedCtl {
   uint64_t item_full[2], item_empty[2];
   uint64_t ring_full[kRing], ring_empty[kRing];
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t k_full[kStages];         // K-side stage loaded (its reuse waits for the S MMA: s_full)
+  uint64_t v_full[kStages];         // V-side stage loaded (its reuse waits for the PV MMA: pv_done)
   uint64_t s_full[3], p_full[3];    // per TMEM S buffer (tile index % 3)
   uint64_t pv_done[3];              // per TMEM S buffer: its PV completed
   uint64_t xchg;                    // softmax warpgroups: partial row max / sum exchange
@@ -339,9 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ctl.k_full[s], 1);
-      mbar_init(&ctl.k_empty[s], 1);
       mbar_init(&ctl.v_full[s], 1);
-      mbar_init(&ctl.v_empty[s], 1);
     }
     mbar_init(&ctl.q_full, 1);
     mbar_init(&ctl.q_empty, 1);
@@ -540,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool kside = (lane == 0);
     if (lane < 2) {
       int stage = 0;
-      uint32_t phase = 0;
+      uint32_t tl = 0;     // tiles loaded
       uint32_t qseq = 0;   // items with tiles seen (K side loads their Q tiles)
       for (uint32_t r = 0;; ++r) {
         if (!ring_get(r, kside ? kPrKDesc : kPrVDesc)) break;
@@ -557,9 +555,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(sQ + cb * CB, &tm_q, &ctl.q_full, cb * 64, 128 * pair, bh);
           ++qseq;
         }
-        uint64_t* empty = kside ? &ctl.k_empty[stage] : &ctl.v_empty[stage];
+        // The stage was last used by tile tl - kStages; it is free once that
+        // tile's S MMA (K side) or PV MMA (V side) has completed, which the
+        // barriers of its TMEM buffer (tl - kStages) % 3 record.
         uint64_t* full = kside ? &ctl.k_full[stage] : &ctl.v_full[stage];
-        if (!wait(empty, phase ^ 1u, kside ? kPrKEmpty : kPrVEmpty)) break;
+        if (tl >= kStages) {
+          const uint32_t tp = tl - kStages;
+          uint64_t* done = kside ? &ctl.s_full[tp % 3u] : &ctl.pv_done[tp % 3u];
+          if (!wait(done, (tp / 3u) & 1u, kside ? kPrKEmpty : kPrVEmpty)) break;
+        }
+        ++tl;
         uint8_t* dst = (kside ? sK : sV) + stage * kTile;
         if (flags & kDescApprox) {
           mbar_arrive_expect_tx(full, (kside ? 2u : 1u) * p.W * D * 2u);
@@ -582,10 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (nblk == 2) tma_load_3d(dst + cb * CB + 8192, map, full, cb * 64, 64 * jb, bh);
           }
         }
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        if (++stage == kStages) stage = 0;
       }
     }
   } else if (warp == 9) {
@@ -642,7 +644,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_ts(tmem + kTmemO, pbase + 8 * kk, vdesc + 128 * kk, idesc_pv, kk == 0 ? acc0 : 1u);
         }
         umma_commit(&ctl.pv_done[b]);
-        umma_commit(&ctl.v_empty[pv.vstage]);
         SA_PROF(prof[kPrMmaIssuePV] += clock64() - tis;)
         return true;
       };
@@ -685,7 +686,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         umma_commit(&ctl.s_full[b]);
-        umma_commit(&ctl.k_empty[kstage]);
         SA_PROF(prof[kPrMmaIssueS] += clock64() - tis;)
         if (++kstage == kStages) {
           kstage = 0;
