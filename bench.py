@@ -290,6 +290,62 @@ def run_ablation(args):
                           "exact_only": {"rel_l2_vs_dense": re, "cosine_vs_dense": ce}}), flush=True)
 
 
+def run_density(args):
+    """Per-row density report (not a bench line): for each beta, the distribution
+    of |S_i| / N over all query blocks of the workload from sol_attn_stats, as a
+    10-bin histogram with mean, quartiles and extremes.  "Sol-Attn: ...",
+    experiments: per-row sparsity of the adaptive threshold (Fig. 7)."""
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_moments_b200 as sa
+    from synth import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    qb, kb, vb = rank_inputs(wl, 0)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = dev(qb), dev(kb), dev(vb)
+    for beta in args.ablation_betas:
+        sa.forward(q, k, v, beta, wl.chunk)
+        counts = sa.stats(wl.B, wl.H, wl.L)
+        dens = (counts.double() / counts.shape[-1]).flatten().cpu().numpy()
+        hist, edges = np.histogram(dens, bins=10, range=(0.0, 1.0))
+        print(json.dumps({"mode": "density", "workload": wl.name, "beta": beta, "rows": int(dens.size),
+                          "mean": float(dens.mean()), "min": float(dens.min()), "max": float(dens.max()),
+                          "quartiles": [float(x) for x in np.quantile(dens, [0.25, 0.5, 0.75])],
+                          "histogram": {"edges": [round(float(e), 2) for e in edges], "counts": hist.tolist()}}),
+              flush=True)
+
+
+def run_chunk_sweep(args):
+    """Chunk-size sweep (not a bench line): the forward at several C, each against
+    the workload's own C: max |difference| of the outputs (C changes only the
+    order of the online-softmax updates, so only rounding) and the time per call.
+    "Sol-Attn: ...", experiments: setup (C affects efficiency, not the output)."""
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_moments_b200 as sa
+    from synth import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    qb, kb, vb = rank_inputs(wl, 0)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = dev(qb), dev(kb), dev(vb)
+    ref = sa.forward(q, k, v, args.beta, wl.chunk).float()
+    for C in args.chunks:
+        for _ in range(2):
+            o = sa.forward(q, k, v, args.beta, C)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(3):
+            o = sa.forward(q, k, v, args.beta, C)
+        t1.record()
+        torch.cuda.synchronize()
+        diff = (o.float() - ref).abs().max().item()
+        print(json.dumps({"mode": "chunk_sweep", "workload": wl.name, "beta": args.beta, "chunk": C,
+                          "ms_per_call": t0.elapsed_time(t1) / 3, "max_abs_diff_vs_default_chunk": diff}),
+              flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -305,7 +361,13 @@ def main():
     ap.add_argument("--no-dense", action="store_true", help="skip the select-all (dense) comparison run")
     ap.add_argument("--ablation", action="store_true",
                     help="approximation ablation: full method and exact-only against select-all (not a bench line)")
-    ap.add_argument("--ablation-betas", type=float, nargs="+", default=[0.75, 1.0, 1.5])
+    ap.add_argument("--ablation-betas", type=float, nargs="+", default=[0.75, 1.0, 1.5],
+                    help="betas of --ablation and --density")
+    ap.add_argument("--chunk-sweep", action="store_true",
+                    help="outputs and times at several chunk sizes C (not a bench line)")
+    ap.add_argument("--chunks", type=int, nargs="+", default=[1, 16, 64, 256, 1024])
+    ap.add_argument("--density", action="store_true",
+                    help="per-row density histogram from sol_attn_stats (not a bench line)")
     ap.add_argument("--role-profile", action="store_true",
                     help="run the profiling build (libsol_attn_profile.so) and print per-role cycle accounting")
     args = ap.parse_args()
@@ -313,6 +375,10 @@ def main():
         return run_role_profile(args)
     if args.ablation:
         return run_ablation(args)
+    if args.density:
+        return run_density(args)
+    if args.chunk_sweep:
+        return run_chunk_sweep(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

@@ -15,7 +15,8 @@
 // blocks reach that half through the approximation instead).  The result is
 // the same as processing the blocks one by one.
 //
-// For each chunk of C pooled keys the item's tile sequence holds
+// For each window of pooled keys (the chunk C, widened to at least 64) the
+// item's tile sequence holds
 //   exact   the selected blocks of the chunk, two per tile: S = Q·[K_a;K_b]ᵀ
 //           (128 x 128), per-half / key >= L masks, online-softmax update,
 //           O += P·[V_a;V_b];
@@ -91,7 +92,7 @@ constexpr unsigned kStatusDevice = 2u;
 
 struct FusedParams {
   int BH, L, N, W;          // W: approximation tile width (MMA N), 32 or 64
-  int chunk;                // C
+  int chunk;                // window of the tile walk: max(C, 64) pooled keys
   int num_pairs, num_items;
   unsigned flags;
   float scale_log2;         // log2(e) / sqrt(d)

@@ -284,7 +284,13 @@ int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void
   const long long BH = static_cast<long long>(s.B) * s.H;
   if ((N + 31) / 32 > kMaxMaskWords)
     return fail(SOL_ATTN_ERR_UNSUPPORTED, "N = %d pooled blocks exceeds the fused kernel's %d", N, kMaxMaskWords * 32);
-  const int W = std::min(64, (std::min(chunk, N) + 31) / 32 * 32);
+  // The tile walk goes through windows of max(C, 64) pooled keys.  The
+  // selection does not depend on C (the union of the chunk-wise selections is
+  // the global one) and the online softmax does not depend on the order of its
+  // tiles, so C only shapes the walk; windows narrower than 64 blocks would
+  // only make the approximation tiles narrower and the exact tiles single-block.
+  const int win = std::max(chunk, 64);
+  const int W = std::min(64, (std::min(win, N) + 31) / 32 * 32);
   CUtensorMap tq, tk, tv, tkb, tkl, tvb;
   int rc;
   if ((rc = make_map(&tq, q, D, s.L, BH, 128))) return rc;
@@ -299,7 +305,7 @@ int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void
   p.L = s.L;
   p.N = N;
   p.W = W;
-  p.chunk = chunk;
+  p.chunk = win;
   p.num_pairs = (N + 1) / 2;
   p.num_items = static_cast<int>(BH * p.num_pairs);
   p.flags = flags;
