@@ -245,16 +245,19 @@ int run_pool(Workspace& w, const void* q, const void* k, const void* v, const so
 template <int D>
 int launch_threshold(Workspace& w, int N, float beta, int mode, const sol_attn_debug* dbg, cudaStream_t st) {
   const int BH = w.shape.B * w.shape.H;
-  moments_kernel<D><<<BH, 256, 0, st>>>(w.kbar, N, w.mom_mean, w.mom_cov);
+  constexpr int T = D / 64;
+  moments_kernel<D><<<dim3(T * (T + 1) / 2, BH), 256, 0, st>>>(w.kbar, N, w.mom_mean, w.mom_cov);
   CUDA_TRY(cudaGetLastError());
-  const size_t smem = (static_cast<size_t>(D) * D + D + 8 * 4 * D) * sizeof(double);
-  static bool attr_set = false;
-  if (!attr_set) {
+  constexpr size_t smem = threshold_smem_bytes(D);
+  static bool attr_set[kMaxDevices] = {false};
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
     CUDA_TRY(cudaFuncSetAttribute(threshold_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(smem)));
-    attr_set = true;
+    attr_set[dev] = true;
   }
-  dim3 grid((N + 31) / 32, BH);
+  dim3 grid((N + kThresholdBlocksPerCta - 1) / kThresholdBlocksPerCta, BH);
   threshold_kernel<D><<<grid, 256, smem, st>>>(w.qbar, w.mom_mean, w.mom_cov, N, beta, mode, w.tau,
                                                 dbg ? dbg->mu : nullptr, dbg ? dbg->sigma : nullptr);
   CUDA_TRY(cudaGetLastError());
