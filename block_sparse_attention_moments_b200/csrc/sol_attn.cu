@@ -511,7 +511,7 @@ int sol_attn_forward_host(const uint16_t* q, const uint16_t* k, const uint16_t* 
   // The (batch, head) slices are independent and contiguous: they go through in
   // up to kHostChunks groups, the copy in of group c + 1 and the copy out of
   // group c - 1 overlapping the kernels of group c.
-  constexpr int kHostChunks = 8;
+  constexpr int kHostChunks = 16;
   const int BH = B * H;
   const int hc = (BH + kHostChunks - 1) / kHostChunks;     // heads per group
   const int ngroups = (BH + hc - 1) / hc;

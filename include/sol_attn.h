@@ -98,7 +98,7 @@ int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out,
 int sol_attn_stats(int32_t* counts, int B, int H, int L, int block, void* stream);
 
 /* End-to-end call on HOST buffers (pinned or pageable; pinned lets the copies
- * overlap): the B*H independent (batch, head) slices go through in up to 8
+ * overlap): the B*H independent (batch, head) slices go through in up to 16
  * groups; for each group q, k, v are copied to the device, sol_attn_forward_ex
  * runs on the group and out is copied back, on three internal streams so that
  * the copies of neighbouring groups overlap the kernels.  Synchronises before
