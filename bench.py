@@ -346,6 +346,56 @@ def run_chunk_sweep(args):
               flush=True)
 
 
+def run_speedup_sweep(args):
+    """Speedup over the kernel's own select-all (dense) mode across sequence
+    lengths and sparsity levels (not a bench line): per length L, bf16
+    Fourier-feature inputs on a (L/4096) x 64 x 64 token grid, `--sweep-heads`
+    heads, d = 128, C = 64; per beta the measured density (sol_attn_stats), the
+    time per forward and the speedup.  L2 is flushed (256 MB write) before every
+    timed call.  "Sol-Attn: ...", experiments: kernel-level speedup over dense
+    attention across 16K-128K tokens and sparsity levels (Fig. 5a)."""
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_moments_b200 as sa
+    from synth import custom_fourier
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
+    H, d, C = args.sweep_heads, 128, 64
+
+    def time_call(fn, reps=3):
+        for _ in range(2):
+            fn()
+        total = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            fn()
+            t1.record()
+            torch.cuda.synchronize()
+            total += t0.elapsed_time(t1)
+        return total / reps
+
+    for L in args.sweep_lengths:
+        qb, kb, vb = custom_fourier(1, H, (max(1, L // 4096), 64, 64), d, 3.0, seed=2000 + L // 1024)
+        q, k, v = dev(qb), dev(kb), dev(vb)
+        Lr = q.shape[2]
+        N = -(-Lr // sa.BLOCK)
+        dense_ms = time_call(lambda: sa.forward(q, k, v, -math.inf, C, flags=sa.FLAG_SELECT_ALL))
+        for beta in args.sweep_betas:
+            ms = time_call(lambda: sa.forward(q, k, v, beta, C))
+            counts = sa.stats(1, H, Lr)
+            pairs = int(counts.to(torch.int64).sum().item())
+            density = pairs / (H * N * N)
+            tflops = sa.executed_flops(pairs, 1, H, Lr, d, approx=True) / (ms * 1e-3) / 1e12
+            print(json.dumps({"mode": "speedup_sweep", "L": Lr, "heads": H, "beta": beta,
+                              "density": round(density, 4), "sparsity": round(1.0 - density, 4),
+                              "ms_per_call": ms, "dense_ms_per_call": dense_ms,
+                              "speedup_vs_dense": dense_ms / ms, "executed_tflops": tflops}), flush=True)
+        del q, k, v
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -368,6 +418,12 @@ def main():
     ap.add_argument("--chunks", type=int, nargs="+", default=[1, 16, 64, 256, 1024])
     ap.add_argument("--density", action="store_true",
                     help="per-row density histogram from sol_attn_stats (not a bench line)")
+    ap.add_argument("--speedup-sweep", action="store_true",
+                    help="speedup over the select-all mode across lengths and sparsity (not a bench line)")
+    ap.add_argument("--sweep-lengths", type=int, nargs="+", default=[16384, 32768, 65536, 131072])
+    ap.add_argument("--sweep-betas", type=float, nargs="+", default=[0.84, 1.28, 1.64],
+                    help="about 80%%, 90%% and 95%% sparsity on Gaussian proxy logits")
+    ap.add_argument("--sweep-heads", type=int, default=8)
     ap.add_argument("--role-profile", action="store_true",
                     help="run the profiling build (libsol_attn_profile.so) and print per-role cycle accounting")
     args = ap.parse_args()
@@ -377,6 +433,8 @@ def main():
         return run_ablation(args)
     if args.density:
         return run_density(args)
+    if args.speedup_sweep:
+        return run_speedup_sweep(args)
     if args.chunk_sweep:
         return run_chunk_sweep(args)
     if args.warmup < 3:
