@@ -34,7 +34,7 @@ from typing import Optional
 import numpy as np
 
 __all__ = [
-    "Workload", "WORKLOADS", "grid_coords", "fourier_inputs", "gauss_inputs",
+    "Workload", "WORKLOADS", "grid_coords", "fourier_inputs", "gauss_inputs", "ramp_inputs",
     "bf16_round", "bf16_bits_to_f64", "f32_to_bf16_bits", "f32_to_bf16_bits_np",
 ]
 
@@ -167,6 +167,19 @@ def gauss_inputs(B: int, H: int, L: int, d: int, seed: int):
     rng = np.random.Generator(np.random.PCG64(seed))
     x = rng.standard_normal(size=(3, B, H, L, d), dtype=np.float32)
     return f32_to_bf16_bits(x[0]), f32_to_bf16_bits(x[1]), f32_to_bf16_bits(x[2])
+
+
+def ramp_inputs(B: int, H: int, L: int, d: int, q_amp: float, k_lo: float, k_hi: float, seed: int,
+                v_amp: float = 1.0):
+    """bf16 Q, K, V bits [B, H, L, d]: Q ~ N(0, q_amp^2), V ~ N(0, v_amp^2), and K ~ N(0, s_t^2)
+    with the scale s_t rising linearly from k_lo (first token) to k_hi (last), so a row's
+    largest logits sit late in the sequence."""
+    rng = np.random.default_rng(seed)
+    s = (k_lo + (k_hi - k_lo) * np.arange(L, dtype=np.float64) / max(L - 1, 1)).astype(np.float32)
+    q = rng.standard_normal((B, H, L, d), dtype=np.float32) * np.float32(q_amp)
+    k = rng.standard_normal((B, H, L, d), dtype=np.float32) * s[None, None, :, None]
+    v = rng.standard_normal((B, H, L, d), dtype=np.float32) * np.float32(v_amp)
+    return f32_to_bf16_bits_np(q), f32_to_bf16_bits_np(k), f32_to_bf16_bits_np(v)
 
 
 def custom_fourier(B: int, H: int, grid, d: int, amp: float, seed: int):

@@ -10,7 +10,7 @@ import pytest
 
 import block_sparse_attention_moments_b200 as sa
 from parity_util import Report, compare_head, debug_numpy, run_gpu
-from synth import WORKLOADS, custom_fourier, fourier_inputs, gauss_inputs
+from synth import WORKLOADS, custom_fourier, fourier_inputs, gauss_inputs, ramp_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -45,11 +45,23 @@ def test_tiny_shape(beta):
     _full_check(qb, kb, vb, beta, wl.chunk)
 
 
-@pytest.mark.parametrize("beta", [0.5, 1.0, 1.5, -math.inf])
+@pytest.mark.parametrize("beta", [0.5, 1.0, 1.5, -math.inf, 0.0, -0.5])
 def test_small_shape(beta):
     wl = WORKLOADS["small"]
     qb, kb, vb = fourier_inputs(wl)
     _full_check(qb, kb, vb, beta, wl.chunk)
+
+
+@pytest.mark.parametrize("beta", [-math.inf, 0.5, 1.0])
+def test_running_maximum_rises_along_the_walk(beta):
+    # Key norms grow along the sequence, so most rows meet their largest logits
+    # late in their walk: the running maximum rises by tens of doublings, and
+    # the rare path (raise m, rescale O, recompute P from S) runs on most rows.
+    # The softmax rows are nearly one-hot here, so O is about one row of V; V is
+    # scaled by 1/4 to keep |O| in the range of the other workloads (with unit V,
+    # |O| reaches 4.9, where one bf16 rounding of the output alone is 0.016).
+    qb, kb, vb = ramp_inputs(1, 2, 4096, 128, 2.0, 0.25, 4.0, seed=91, v_amp=0.25)
+    _full_check(qb, kb, vb, beta, 16)
 
 
 def test_chunk_size_does_not_change_the_result():
