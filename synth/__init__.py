@@ -34,7 +34,7 @@ from typing import Optional
 import numpy as np
 
 __all__ = [
-    "Workload", "WORKLOADS", "grid_coords", "fourier_inputs", "gauss_inputs", "ramp_inputs",
+    "Workload", "WORKLOADS", "grid_coords", "fourier_inputs", "gauss_inputs", "ramp_inputs", "offset_inputs",
     "bf16_round", "bf16_bits_to_f64", "f32_to_bf16_bits", "f32_to_bf16_bits_np",
 ]
 
@@ -179,6 +179,18 @@ def ramp_inputs(B: int, H: int, L: int, d: int, q_amp: float, k_lo: float, k_hi:
     q = rng.standard_normal((B, H, L, d), dtype=np.float32) * np.float32(q_amp)
     k = rng.standard_normal((B, H, L, d), dtype=np.float32) * s[None, None, :, None]
     v = rng.standard_normal((B, H, L, d), dtype=np.float32) * np.float32(v_amp)
+    return f32_to_bf16_bits_np(q), f32_to_bf16_bits_np(k), f32_to_bf16_bits_np(v)
+
+
+def offset_inputs(B: int, H: int, L: int, d: int, a: float, sign: float, noise: float, seed: int):
+    """bf16 Q, K, V bits [B, H, L, d] whose logits all sit near sign * a^2 / sqrt(d):
+    Q = a e_0 + noise N(0, I), K = sign a e_0 + noise N(0, I), V ~ N(0, 1)."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, H, L, d), dtype=np.float32) * np.float32(noise)
+    k = rng.standard_normal((B, H, L, d), dtype=np.float32) * np.float32(noise)
+    q[..., 0] += np.float32(a)
+    k[..., 0] += np.float32(sign * a)
+    v = rng.standard_normal((B, H, L, d), dtype=np.float32)
     return f32_to_bf16_bits_np(q), f32_to_bf16_bits_np(k), f32_to_bf16_bits_np(v)
 
 

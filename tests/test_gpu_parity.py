@@ -10,7 +10,7 @@ import pytest
 
 import block_sparse_attention_moments_b200 as sa
 from parity_util import Report, compare_head, debug_numpy, run_gpu
-from synth import WORKLOADS, custom_fourier, fourier_inputs, gauss_inputs, ramp_inputs
+from synth import WORKLOADS, custom_fourier, fourier_inputs, gauss_inputs, offset_inputs, ramp_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -62,6 +62,17 @@ def test_running_maximum_rises_along_the_walk(beta):
     # |O| reaches 4.9, where one bf16 rounding of the output alone is 0.016).
     qb, kb, vb = ramp_inputs(1, 2, 4096, 128, 2.0, 0.25, 4.0, seed=91, v_amp=0.25)
     _full_check(qb, kb, vb, beta, 16)
+
+
+@pytest.mark.parametrize("sign", [-1.0, 1.0])
+@pytest.mark.parametrize("beta", [-math.inf, 1.0])
+def test_logits_far_from_zero(sign, beta):
+    # Every logit near -141 (or +141) nats, about -204 (+204) doublings: against
+    # the provisional reference 0 of a row's first tile every 2^y underflows to
+    # 0 (or overflows to inf), so the row's first m must come from its exact
+    # maximum; softmax is shift-invariant, so the result is ordinary attention.
+    qb, kb, vb = offset_inputs(1, 2, 2048, 128, 40.0, sign, 0.1, seed=93)
+    _full_check(qb, kb, vb, beta, 8)
 
 
 def test_chunk_size_does_not_change_the_result():
