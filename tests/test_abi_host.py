@@ -64,6 +64,9 @@ def test_workspace_size_is_host_arithmetic(lib):
     got = sa.workspace_bytes(B, H, L, d)
     assert expect_min <= got <= expect_min + 64 * 1024 * 1024
     assert sa.workspace_bytes(1, 1, 128, 96) == 0
+    # the longest sequence is 2^20 tokens (16384 pooled blocks, the fused kernel's mask capacity)
+    assert sa.workspace_bytes(1, 1, 1 << 20, 64) > 0
+    assert sa.workspace_bytes(1, 1, (1 << 20) + 1, 64) == 0
     assert sa.kernels_per_forward() == 4
 
 

@@ -135,6 +135,13 @@ def test_edge_shapes(L, d, chunk, beta):
     _full_check(qb, kb, vb, beta, chunk)
 
 
+def test_maximum_length_sampled():
+    # The longest sequence accepted: L = 2^20, N = 16384 pooled blocks, 512 mask
+    # words per row; one head, sampled query blocks including the first and last.
+    qb, kb, vb = gauss_inputs(1, 1, 1 << 20, 64, seed=17)
+    _full_check(qb, kb, vb, 1.5, 64, rows=[0, 1, 5000, 12345, 16382, 16383])
+
+
 def test_gaussian_inputs_density():
     qb, kb, vb = gauss_inputs(1, 2, 64 * 512, 128, seed=12)
     for beta, rho in ((0.5, 0.3085), (1.0, 0.1587), (1.5, 0.0668)):
