@@ -249,9 +249,10 @@ int launch_threshold(Workspace& w, int N, float beta, int mode, const sol_attn_d
   moments_kernel<D><<<dim3(T * (T + 1) / 2, BH), 256, 0, st>>>(w.kbar, N, w.mom_mean, w.mom_cov);
   CUDA_TRY(cudaGetLastError());
   constexpr size_t smem = threshold_smem_bytes(D);
-  static bool attr_set[kMaxDevices] = {false};
+  static bool attr_set[kMaxDevices] = {false};   // the attribute is set per device
   int dev = 0;
   CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(SOL_ATTN_ERR_UNSUPPORTED, "device index %d too large", dev);
   if (!attr_set[dev]) {
     CUDA_TRY(cudaFuncSetAttribute(threshold_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(smem)));
@@ -331,11 +332,12 @@ int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void
   int dev = 0, nsm = 0;
   CUDA_TRY(cudaGetDevice(&dev));
   CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
-  static bool attr_set = false;
-  if (!attr_set) {
+  static bool attr_set[kMaxDevices] = {false};   // the attribute is set per device
+  if (dev < 0 || dev >= kMaxDevices) return fail(SOL_ATTN_ERR_UNSUPPORTED, "device index %d too large", dev);
+  if (!attr_set[dev]) {
     CUDA_TRY(cudaFuncSetAttribute(sol_attn_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(kFusedSmemBytes)));
-    attr_set = true;
+    attr_set[dev] = true;
   }
   CUDA_TRY(cudaMemsetAsync(w.counter, 0, sizeof(unsigned), st));
   const int grid = std::min(p.num_items, nsm);
