@@ -246,3 +246,41 @@ def test_sel_override_reproduces_threshold_selection():
     a = sol_attn_head(q, k, v, 1.0)
     b = sol_attn_head(q, k, v, 1.0, sel_override=a["sel"])
     np.testing.assert_array_equal(a["O"], b["O"])
+
+
+# --- output structure (method: Eq. 9-10, the normalised sum over exact and approximated keys) ---
+
+@pytest.mark.parametrize("beta", [0.5, 1.0, math.inf])
+def test_constant_values_give_that_constant(beta):
+    # With V = c everywhere, V̂_j = n_j c, so every output row is
+    # (Σ e^s c + Σ_j n_j e^a c) / (Σ e^s + Σ_j n_j e^a) = c exactly: the weights
+    # are normalised, and n_j appears on both sides (a ragged 37-token tail
+    # included).  Dropping n_j from either side, or pooling V̂ as a mean, breaks it.
+    q, k, _ = _fourier_head((1, 1, 64 * 9 + 37), 64, seed=41)
+    c = np.array([0.75, -2.5] * 32)
+    v = np.tile(c, (q.shape[0], 1))
+    out = sol_attn_head(q, k, v, beta)["O"]
+    np.testing.assert_allclose(out, np.tile(c, (q.shape[0], 1)), rtol=0, atol=1e-12)
+
+
+def test_output_is_linear_in_values():
+    # The selection and every weight depend on Q and K only, so the output is
+    # linear in V (V̂ is a linear pooling of V).
+    q, k, v1 = _fourier_head((1, 2, 300), 64, seed=43)
+    v2 = np.random.default_rng(2).normal(size=v1.shape)
+    for beta in (0.5, 1.0):
+        o1 = sol_attn_head(q, k, v1, beta)["O"]
+        o2 = sol_attn_head(q, k, v2, beta)["O"]
+        o12 = sol_attn_head(q, k, 2.0 * v1 - 0.5 * v2, beta)["O"]
+        np.testing.assert_allclose(o12, 2.0 * o1 - 0.5 * o2, rtol=0, atol=1e-10)
+
+
+def test_query_key_rescaling_invariance():
+    # (Q, K) -> (c Q, K / c) leaves every exact, proxy and approximation logit
+    # unchanged, and with them μ_i, σ_i, τ_i: same selection, same output.
+    q, k, v = _fourier_head((2, 8, 50), 64, seed=47)
+    for beta in (0.5, 1.0):
+        a = sol_attn_head(q, k, v, beta)
+        b = sol_attn_head(4.0 * q, k / 4.0, v, beta)
+        np.testing.assert_array_equal(a["sel"], b["sel"])
+        np.testing.assert_allclose(a["O"], b["O"], rtol=0, atol=1e-10)
