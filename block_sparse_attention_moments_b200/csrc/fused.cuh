@@ -160,6 +160,7 @@ constexpr uint32_t kSmemK = kSmemQ + kTile;
 constexpr uint32_t kSmemV = kSmemK + kStages * kTile;
 constexpr uint32_t kSmemCtl = kSmemV + kStages * kTile;
 constexpr uint32_t kFusedSmemBytes = kSmemCtl + sizeof(FusedCtl) + 1024;  // + alignment slack
+static_assert(kFusedSmemBytes <= 227u * 1024u, "dynamic shared memory of one CTA on sm_100");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0, kTmemS0 = 128;    // O at [0, 128), S / P buffer b at 128 + 128 b (b < 3)
 constexpr int kThreads = 384;
