@@ -457,8 +457,14 @@ def main():
     q, k, v = dev(qb), dev(kb), dev(vb)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
+    in_bytes = 3 * B * H * L * d * 2
+    # inputs that fit in L2 are evicted by a 256 MB write before every timed step
+    # (outside the stage events, which then give the step time)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda") if in_bytes <= (126 << 20) else None
 
     def step(beta, flags, ev=None):
+        if flush is not None:
+            flush.zero_()
         if ev is None:
             sa.stage_pool(q, k, v, stream=stream)
             sa.stage_threshold(B, H, L, d, beta, flags=flags, stream=stream)
@@ -494,6 +500,8 @@ def main():
             pg.barrier()
         total_ms = start.elapsed_time(end)
         per = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(3)]
+        if flush is not None:   # the flushes sit between the steps: time the stages only
+            total_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
         counts = sa.stats(B, H, L, stream=stream)
         torch.cuda.synchronize()
         pairs = int(counts.to(torch.int64).sum().item())
@@ -562,7 +570,9 @@ def main():
         "config": {"workload": f"{wl.name}: {WORKLOAD_TEXT.get(wl.name, wl.name)} per GPU, block=64 C={C} "
                                f"beta={args.beta}, bf16 Fourier-feature Q/K, Gaussian V",
                    "per_gpu_batch": 1, "global_batch": world, "seq_len": L, "parallelism": f"dp{world} (weak)",
-                   "l2": "inputs (2.3 GB/step) larger than L2 (126 MB)"},
+                   "l2": (f"inputs ({in_bytes / 1e9:.2f} GB/step) larger than L2 (126 MB)" if flush is None else
+                          f"inputs ({in_bytes / 1e6:.1f} MB/step) fit in L2: a 256 MB write flushes it before "
+                          f"each step, outside the timed stages")},
         "ms_per_call": step_ms,
         "pct_bf16_peak": 100.0 * value / world / peak,
         "stage_ms": {"pool": per_ms[0], "threshold": per_ms[1], "fused": per_ms[2]},
@@ -572,7 +582,9 @@ def main():
         sa.executed_flops(dense_pairs, B, H, L, d, approx=False) / (dense_step_ms * 1e-3) / 1e12,
         "speedup_vs_dense": None if args.no_dense else dense_step_ms / step_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": load_traffic(),
+                     "frac": achieved / peak,
+                     # the committed capture covers the default workload's sparse call only
+                     "traffic": load_traffic() if (wl.name == "wan" and args.beta == 1.0) else None,
                      "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"
                      else "fallback 1.59 PFLOP/s", "frac_of_sustained": achieved / peak_sus,
                      "kernel": "sol_attn_fused_kernel", "algorithmic_flops_per_launch": fused_flops},
