@@ -26,6 +26,12 @@ reading is listed in the design notes:
         O_r = N_r / D_r        (0 when D_r = 0, which only exact-only can reach).
     The approximation uses the per-token logit q_r·K̄_j (the B x 1 centre of the
     zeroth-order Taylor term), not the block-level ŝ_ij.
+  * optional first-order term (taylor_order=1): the expansion of a skipped
+    block's exponential scores around that same centre c_r = q_r·K̄_j/sqrt(d),
+        exp(s_rk) ≈ exp(c_r) (1 + (s_rk - c_r)),
+    whose added term exp(c_r)(s_rk - c_r) enters D and N like an exact score
+    (its row sum over the block is zero, so only N changes).  The pages keep
+    the zeroth order only; the first order is this build's extension.
 
 Every array is float64.  Matmuls and reductions are library primitives; there
 is no blocking, fusion or reordering beyond the definitions above.
@@ -40,7 +46,7 @@ import numpy as np
 __all__ = [
     "pool_blocks", "proxy_row", "proxy_logits", "key_moments", "row_stats_from_moments",
     "row_stats_bruteforce", "thresholds", "select_global", "select_streaming",
-    "approx_logits", "sol_attn_head", "sol_attn", "dense_attention_head",
+    "approx_logits", "sol_attn_head",
 ]
 
 
@@ -141,7 +147,8 @@ def approx_logits(q_rows: np.ndarray, kbar: np.ndarray) -> np.ndarray:
 
 
 def sol_attn_head(q, k, v, beta: float, block: int = 64, *, exact_only: bool = False,
-                  rows: Optional[list] = None, sel_override: Optional[np.ndarray] = None):
+                  rows: Optional[list] = None, sel_override: Optional[np.ndarray] = None,
+                  taylor_order: int = 0):
     """Sol-Attn forward for one (batch, head) slice, non-streaming, in fp64.
 
     q, k, v: [L, d] float64 (callers widen the bf16 inputs exactly).
@@ -151,6 +158,8 @@ def sol_attn_head(q, k, v, beta: float, block: int = 64, *, exact_only: bool = F
     threshold test (to evaluate a different but equally valid selection).
     exact_only: keep-or-drop sparse attention on the same selection
     (ablation: exact-only vs exact-or-approx, Fig. 7).
+    taylor_order: 0 (the method: zeroth-order term of Eq. 8) or 1 (adds the
+    first-order term of the same expansion for every unselected block).
 
     Returns dict with O [L, d], counts [N], sel [N, N] (rows evaluated),
     qbar, kbar, vhat, n, mu, sigma, tau.
@@ -200,29 +209,15 @@ def sol_attn_head(q, k, v, beta: float, block: int = 64, *, exact_only: bool = F
         pa = np.exp(a - M)
         D = pe.sum(axis=1) + (pa * n[U][None, :]).sum(axis=1)
         Nn = pe @ v[key_idx] + pa @ vhat[U]
+        if taylor_order >= 1:
+            # first-order term exp(c)(S_j - c) of each skipped block j, with the
+            # block's exact scores S_j and the centre c = a[:, u] broadcast over keys
+            for u, j in enumerate(U):
+                kj = np.arange(j * block, min((j + 1) * block, L))
+                resid = qi @ k[kj].T * scale - a[:, u:u + 1]
+                term = pa[:, u:u + 1] * resid
+                D = D + term.sum(axis=1)
+                Nn = Nn + term @ v[kj]
         O[lo:hi] = Nn / D[:, None]
     return dict(O=O, counts=counts, sel=sel, qbar=qbar, kbar=kbar, vhat=vhat, n=n,
                 mu=mu, sigma=sigma, tau=tau, m=m, sigma_k=sigma_k)
-
-
-def sol_attn(q, k, v, beta: float, block: int = 64, *, exact_only: bool = False):
-    """Batched form over [B, H, L, d]; returns (O [B,H,L,d], counts [B,H,N], sel [B,H,N,N])."""
-    B, H, L, d = q.shape
-    N = _nblocks(L, block)
-    O = np.zeros((B, H, L, d))
-    counts = np.zeros((B, H, N), dtype=np.int64)
-    sel = np.zeros((B, H, N, N), dtype=bool)
-    for b in range(B):
-        for h in range(H):
-            r = sol_attn_head(q[b, h], k[b, h], v[b, h], beta, block, exact_only=exact_only)
-            O[b, h], counts[b, h], sel[b, h] = r["O"], r["counts"], r["sel"]
-    return O, counts, sel
-
-
-def dense_attention_head(q, k, v) -> np.ndarray:
-    """Textbook softmax attention softmax(q k^T / sqrt(d)) v in fp64."""
-    d = q.shape[1]
-    s = q @ k.T / math.sqrt(d)
-    s = s - s.max(axis=1, keepdims=True)
-    p = np.exp(s)
-    return (p @ v) / p.sum(axis=1, keepdims=True)

@@ -31,6 +31,10 @@ MUTANTS = {
     "threshold_minus_beta": ("return mu + beta * sigma", "return mu - beta * sigma"),
     "approx_block_level_logit": ("a = approx_logits(qi, kbar[U])",
                                  "a = np.repeat(approx_logits(qbar[i:i+1], kbar[U]), qi.shape[0], axis=0)"),
+    "first_order_sign": ("term = pa[:, u:u + 1] * resid", "term = -pa[:, u:u + 1] * resid"),
+    "first_order_block_level_centre": ("resid = qi @ k[kj].T * scale - a[:, u:u + 1]",
+                                       "resid = qi @ k[kj].T * scale - proxy_row(qbar[i], kbar[j:j + 1])[None, :]"),
+    "first_order_dropped_from_numerator": ("Nn = Nn + term @ v[kj]", "Nn = Nn"),
 }
 
 

@@ -284,3 +284,57 @@ def test_query_key_rescaling_invariance():
         b = sol_attn_head(4.0 * q, k / 4.0, v, beta)
         np.testing.assert_array_equal(a["sel"], b["sel"])
         np.testing.assert_allclose(a["O"], b["O"], rtol=0, atol=1e-10)
+
+
+# --- first-order term of the expansion (method: proxy-score reuse, Eq. 8; the pages keep
+# --- only the zeroth order, the first order is this build's extension) -----------------
+
+def _blocky_keys(L, d, seed, eps):
+    """Keys equal to their block's mean plus eps times a fixed zero-mean-per-block residual."""
+    q, k, v = _fourier_head((1, 1, L), d, amp=2.5, seed=seed)
+    kbar, _, n = pool_blocks(k)
+    noise = np.random.default_rng(seed + 1).standard_normal(k.shape)
+    for j in range(len(n)):
+        sl = slice(64 * j, 64 * j + n[j])
+        noise[sl] -= noise[sl].mean(axis=0)
+    return q, np.repeat(kbar, n, axis=0), noise, v
+
+
+@pytest.mark.parametrize("beta", [0.5, 1.0, 1.5])
+def test_first_order_error_falls_with_the_square_of_the_key_spread(beta):
+    # With keys K̄_j + eps R (R zero-mean within each block) the skipped blocks'
+    # scores deviate from the centre by O(eps).  Dropping everything after the
+    # zeroth order leaves an O(eps) error in the numerator; keeping the first
+    # order leaves O(eps^2).  Halving eps must halve the first error and quarter
+    # the second (a missing, mis-signed or mis-centred first-order term fails).
+    q, base, noise, v = _blocky_keys(64 * 12 + 37, 64, 19, 0.0)
+    errs = {}
+    for eps in (0.1, 0.05):
+        kk = base + eps * noise
+        dense = _sdpa(q, kk, v)
+        for order in (0, 1):
+            errs[order, eps] = _rel_l2(sol_attn_head(q, kk, v, beta, taylor_order=order)["O"], dense)
+    r0 = errs[0, 0.1] / errs[0, 0.05]
+    r1 = errs[1, 0.1] / errs[1, 0.05]
+    assert 1.8 < r0 < 2.25, r0
+    assert 3.6 < r1 < 4.4, r1
+    assert errs[1, 0.05] < errs[0, 0.05] / 4
+
+
+@pytest.mark.parametrize("L", [1024, 1000])
+def test_first_order_term_vanishes_on_block_constant_keys(L):
+    # Keys equal to their block mean: every score of a skipped block equals its
+    # centre, the first-order term is zero and the output is dense attention.
+    q, k, v = _fourier_head((1, 1, L), 64, amp=2.5, seed=19)
+    kbar, _, n = pool_blocks(k)
+    kc = np.repeat(kbar, n, axis=0)
+    dense = _sdpa(q, kc, v)
+    for beta in (0.0, 1.0, math.inf):
+        r = sol_attn_head(q, kc, v, beta, taylor_order=1)
+        np.testing.assert_allclose(r["O"], dense, rtol=0, atol=1e-12)
+
+
+def test_first_order_with_every_block_selected_is_softmax_attention():
+    q, k, v = _fourier_head((1, 1, 1000), 64)
+    r = sol_attn_head(q, k, v, -math.inf, taylor_order=1)
+    np.testing.assert_allclose(r["O"], _sdpa(q, k, v), rtol=0, atol=1e-12)
