@@ -247,11 +247,17 @@ def run_role_profile(args):
         per_cta = {k2: v2 / nsm for k2, v2 in prof.items()}
         print(json.dumps({"workload": wl.name, "mode": tag, "ctas": nsm, "tiles_per_cta": tiles / nsm,
                           "cycles_per_cta": {k2: round(v2) for k2, v2 in per_cta.items()},
-                          "softmax_cycles_per_tile": {k2: round(prof[k2] / tiles, 1) for k2 in
-                                                      ("softmax.wait_desc", "softmax.pass1",
-                                                       "softmax.rescale", "softmax.pass2", "softmax.epilogue",
-                                                       "softmax.wait_s", "softmax.wait_o",
-                                                       "softmax.wait_exchange")}}), flush=True)
+                          # per tile of the owning warpgroup (each warpgroup takes every other tile)
+                          "softmax_cycles_per_own_tile": {k2: round(prof[k2] / tiles, 1) for k2 in
+                                                          ("softmax.wait_desc", "softmax.wait_s", "softmax.pass",
+                                                           "softmax.wait_handoff", "softmax.meet",
+                                                           "softmax.wait_o", "softmax.epilogue",
+                                                           "softmax.wait_exchange", "softmax.tmem_load",
+                                                           "softmax.exp_block")},
+                          "issuer_cycles_per_tile": {k2: round(prof[k2] / tiles, 1) for k2 in
+                                                     ("s.issue", "s.wait_buffer", "s.wait_k", "s.wait_desc",
+                                                      "pv.issue", "pv.wait_p", "pv.wait_v", "pv.wait_desc")},
+                          "rescales": prof["softmax.rescales"]}), flush=True)
 
 
 def run_ablation(args):

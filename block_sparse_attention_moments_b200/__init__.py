@@ -17,7 +17,7 @@ import os
 from typing import Optional
 
 __all__ = [
-    "FLAG_SELECT_ALL", "FLAG_EXACT_ONLY", "FLAG_SYNC_CHECK", "SolAttnError", "lib", "lib_path",
+    "FLAG_SELECT_ALL", "FLAG_EXACT_ONLY", "FLAG_SYNC_CHECK", "FLAG_TEST_STALL", "SolAttnError", "lib", "lib_path",
     "forward", "stats", "forward_host", "stage_pool", "stage_threshold", "stage_fused",
     "workspace_bytes", "release", "kernels_per_forward", "DebugBuffers", "EXPORTED_SYMBOLS",
     "executed_flops", "BLOCK",
@@ -26,6 +26,7 @@ __all__ = [
 FLAG_SELECT_ALL = 0x1
 FLAG_EXACT_ONLY = 0x2
 FLAG_SYNC_CHECK = 0x4
+FLAG_TEST_STALL = 0x8   # failure-path test only: every bounded device wait runs out (see sol_attn.h)
 BLOCK = 64
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -220,14 +221,17 @@ def workspace_bytes(B: int, H: int, L: int, d: int) -> int:
     return int(lib().sol_attn_workspace_bytes(B, H, L, d, BLOCK))
 
 
+# Slot names of the profiling build's counters, in the order of the ProfSlot
+# enum in csrc/fused.cuh.
 PROFILE_SLOTS = (
     "route.wait_item_empty", "k.wait_desc", "k.wait_q_empty", "k.wait_stage", "v.wait_desc", "v.wait_stage",
-    "mma.wait_p", "mma.wait_v", "mma.wait_desc", "mma.wait_q", "mma.wait_s_empty", "mma.wait_k",
-    "softmax.wait_desc", "softmax.wait_s", "softmax.wait_o", "softmax.wait_exchange",
-    "total.route", "total.k", "total.v", "total.mma", "total.softmax",
-    "softmax.pass1", "softmax.rescale", "softmax.pass2", "softmax.epilogue", "softmax.tiles", "softmax.rescales",
-    "sched.wait_item", "sched.wait_ring", "total.sched", "softmax.redos",
-    "mma.issue_s", "mma.issue_pv",
+    "s.wait_desc", "s.wait_q", "s.wait_buffer", "s.wait_k", "s.issue",
+    "pv.wait_desc", "pv.wait_p", "pv.wait_v", "pv.issue",
+    "softmax.wait_desc", "softmax.wait_s", "softmax.wait_handoff", "softmax.wait_o", "softmax.wait_exchange",
+    "softmax.pass", "softmax.meet", "softmax.epilogue", "softmax.tiles", "softmax.rescales",
+    "sched.wait_item", "sched.wait_ring",
+    "total.route", "total.k", "total.v", "total.s", "total.pv", "total.softmax", "total.sched",
+    "softmax.tmem_load", "softmax.exp_block",
 )
 
 

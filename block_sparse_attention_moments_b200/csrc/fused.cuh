@@ -29,26 +29,39 @@
 // The walk starts at the chunk holding the item's own query blocks (see
 // TileIter).  Epilogue: O / l in bf16 for rows < L.
 //
-// Warp roles (384 threads, one persistent CTA per SM, atomic work counter):
-//   warps 0-7  softmax, two warpgroups: each thread owns one tile row and one
-//              half of every tile's columns; masks, lazy-rescaled one-pass
-//              online softmax, P into TMEM, epilogue.
+// Warp roles (416 threads, one persistent CTA per SM, atomic work counter):
+//   warps 0-7  softmax, two warpgroups that take the tiles in turns (tile t
+//              belongs to warpgroup t & 1); the thread of TMEM lane r owns row
+//              r of its warpgroup's tiles, all columns: row maximum, the
+//              lazy-rescale decision, P = 2^(y - m) into TMEM, row sums.
 //   warp 8     TMA producers: lane 0 loads Q and the K side (K blocks, or K̄
 //              hi/lo), lane 1 the V side (V blocks, or V̄).
-//   warp 9     tcgen05 MMA issuer: S runs up to two tiles ahead of the PVs.
+//   warp 9     tcgen05 issuer of the S MMAs (up to three tiles in flight).
 //   warp 10    routing: fetches the next item, computes ŝ_ij = Q̄_i·K̄_j/sqrt(d)
 //              in fp32 for both halves, compares with τ_i (warp ballot -> mask
 //              words), one item ahead (double-buffered mask slots).
 //   warp 11    scheduler: walks each item's tile sequence from its masks and
 //              publishes one descriptor per tile (blocks, column validity per
 //              half, first/last flags) into a shared-memory ring that the
-//              producers, the MMA issuer and the softmax warps consume.
+//              producers, both MMA issuers and the softmax warps consume.
+//   warp 12    tcgen05 issuer of the PV MMAs (O += P·V, in tile order).
+// S and PV have an issuer each: an MMA occupies its issuing thread for about
+// its execution time, so one thread alternating between waiting for P and
+// issuing leaves the tensor pipe idle between the two batches.
 //
-// The two threads of a row (one per warpgroup) share one reference maximum,
-// agreed per tile through shared memory, so a single O accumulates the whole
-// row.  P is written back into TMEM over the thread's own part of its S tile
-// (bf16 pairs) and fed to the PV MMA as its A operand, so the only
-// shared-memory operand traffic is Q, K and V.
+// Both warpgroups accumulate into one O per row, so they share the row's
+// reference maximum m (log2 units, a whole number).  The owner of tile t
+// computes P in one pass over its row, 32 columns at a time, against the m
+// its own previous tile of the item settled on, raising it (lazy rescale)
+// only when a group's maximum exceeds it by more than 8 (the groups already
+// stored are scaled by the exact power of two).  At the end of the tile it
+// meets the m that tile t - 1 settled on (shared memory, one mbarrier per
+// hand-off slot): the larger wins, and this tile's P or O (after PV(t - 1)
+// has completed), whichever is behind, is scaled by 2^-k.  Each thread keeps
+// its partial row sum with the m it was accumulated at, and the two partials
+// meet in the epilogue.  P is written back into TMEM over the consumed
+// columns of its S tile (bf16 pairs) and fed to the PV MMA as its A operand,
+// so the only shared-memory operand traffic is Q, K and V.
 //
 // Shared memory (1024-byte aligned, 128-byte swizzled tiles):
 //   Q 32 KB | K ring 2 x 32 KB | V ring 2 x 32 KB | control.
@@ -71,11 +84,11 @@ constexpr int kMaxMaskWords = 512;       // N <= 16384 pooled blocks per head
 // the per-CTA totals are summed into g_profile at exit.
 enum ProfSlot : int {
   kPrRouteWait, kPrKDesc, kPrKQEmpty, kPrKEmpty, kPrVDesc, kPrVEmpty,
-  kPrMmaP, kPrMmaV, kPrMmaDesc, kPrMmaQ, kPrMmaSEmpty, kPrMmaK,
-  kPrSmDesc, kPrSmS, kPrSmO, kPrSmX,
-  kPrTotRoute, kPrTotK, kPrTotV, kPrTotMma, kPrTotSm,
-  kPrSmPass1, kPrSmRescale, kPrSmPass2, kPrSmEpi, kPrSmTiles, kPrSmRescales, kPrSchedItem, kPrSchedRing,
-  kPrTotSched, kPrSmRedo, kPrMmaIssueS, kPrMmaIssuePV, kPrSlots
+  kPrSDesc, kPrSQ, kPrSBuf, kPrSK, kPrSIssue,
+  kPrPvDesc, kPrPvP, kPrPvV, kPrPvIssue,
+  kPrSmDesc, kPrSmS, kPrSmHand, kPrSmO, kPrSmX, kPrSmPass, kPrSmMeet, kPrSmEpi, kPrSmTiles, kPrSmRescales,
+  kPrSchedItem, kPrSchedRing,
+  kPrTotRoute, kPrTotK, kPrTotV, kPrTotS, kPrTotPv, kPrTotSm, kPrTotSched, kPrSmLd, kPrSmExp, kPrSlots
 };
 constexpr int kProfileSlots = 48;
 static_assert(kPrSlots <= kProfileSlots, "profile slots");
@@ -87,8 +100,9 @@ __device__ unsigned long long g_profile[kProfileSlots];
 #endif
 constexpr unsigned kFlagSelectAll = 1u;
 constexpr unsigned kFlagExactOnly = 2u;
+constexpr unsigned kFlagTestStall = 8u;    // routing publishes nothing: every role's wait runs out
 constexpr unsigned kStatusTimeout = 1u;
-constexpr unsigned kStatusDevice = 2u;
+constexpr unsigned kStatusDevice = 2u;     // a tile descriptor failed its range check
 
 struct FusedParams {
   int BH, L, N, W;          // W: approximation tile width (MMA N), 32 or 64
@@ -137,8 +151,10 @@ struct __align__(16) ItemSlot {
 
 struct __align__(16) FusedCtl {
   ItemSlot slot[2];
-  TileDesc ring[kRing];             // scheduler -> producers, MMA issuer, softmax
+  TileDesc ring[kRing];             // scheduler -> producers, MMA issuers, softmax
   float qbar[2][128];               // routing: pooled queries of the pair
+  float hand[3][128];               // [tile % 3][row]: the m tile t settled on, read by tile t + 1
+  float2 xval[2][2][128];           // epilogue: [parity][warpgroup][row] partial (row sum, its m)
   uint64_t item_full[2], item_empty[2];
   uint64_t ring_full[kRing], ring_empty[kRing];
   uint64_t q_full, q_empty;
@@ -146,8 +162,8 @@ struct __align__(16) FusedCtl {
   uint64_t v_full[kStages];         // V-side stage loaded (its reuse waits for the PV MMA: pv_done)
   uint64_t s_full[3], p_full[3];    // per TMEM S buffer (tile index % 3)
   uint64_t pv_done[3];              // per TMEM S buffer: its PV completed
-  uint64_t xchg;                    // softmax warpgroups: partial row max / sum exchange
-  float xval[2][2][128];            // [phase parity][warpgroup][row]
+  uint64_t mready[3];               // per TMEM S buffer: hand[] of that tile written
+  uint64_t xchg;                    // softmax warpgroups: epilogue exchange
   uint32_t tmem_base;
   int abort;
 };
@@ -163,9 +179,13 @@ constexpr uint32_t kFusedSmemBytes = kSmemCtl + sizeof(FusedCtl) + 1024;  // + a
 static_assert(kFusedSmemBytes <= 227u * 1024u, "dynamic shared memory of one CTA on sm_100");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0, kTmemS0 = 128;    // O at [0, 128), S / P buffer b at 128 + 128 b (b < 3)
-constexpr int kThreads = 384;
-constexpr int kSoftmaxThreads = 256;   // two warpgroups, each owning half of every tile's columns
-constexpr uint32_t kRingEmptyCount = 8 + 3;  // softmax warps (lane 0 each) + K producer + V producer + MMA
+constexpr int kThreads = 416;                    // 13 warps
+// Registers: the 13 warps sit 4-3-3-3 on the SM's four sub-partitions, each
+// with a quarter of the register file, so a thread may hold at most 128.
+constexpr int kLaunchBoundThreads = 512;
+constexpr int kWarpLoad = 8, kWarpS = 9, kWarpRoute = 10, kWarpSched = 11, kWarpPv = 12;
+constexpr uint32_t kRingEmptyCount = 8 + 4;      // softmax warps (lane 0 each) + K, V producers + S, PV issuers
+constexpr uint32_t kPFullCount = 8;              // owner warps arrive 2 each; on an item's first tile all 8 arrive 1
 
 __device__ __forceinline__ bool mask_bit(const uint32_t* m, int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
 
@@ -303,8 +323,47 @@ __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile 
   return false;
 }
 
+// Largest of 32 values (three-input max, a tree of depth 4).
+__device__ __forceinline__ float max32(const float* x) {
+  float a[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) a[i] = max3f(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+  a[10] = fmaxf(x[30], x[31]);
+  const float b0 = max3f(a[0], a[1], a[2]), b1 = max3f(a[3], a[4], a[5]), b2 = max3f(a[6], a[7], a[8]);
+  return max3f(max3f(b0, b1, b2), a[9], a[10]);
+}
+
+// Multiplies the bf16 P values already stored in the first n 16-column groups
+// of a row's S/P buffer by f (a power of two: exact).  Warp-wide.
+__device__ __noinline__ void scale_p(uint32_t tS, int n, float f) {
+  tmem_st_wait();   // the groups' stores have landed
+  const __nv_bfloat162 f2 = __floats2bfloat162_rn(f, f);
+#pragma unroll 1
+  for (int g = 0; g < n; ++g) {
+    float r[16];
+    tmem_ld_x16f(tS + 16 * g, r);
+    tmem_ld_wait();
+    reg_fence16(r);
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&r[e]);
+      h = __hmul2(h, f2);
+      w[e] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    tmem_st_x16(tS + 16 * g, w);
+  }
+}
+
+// 2^-k for a whole number k >= 0 given as a float difference of two whole
+// numbers (0 below the fp32 range), exact.
+__device__ __forceinline__ float exp2_neg_int(float k) {
+  const int ki = __float2int_rn(k);
+  return (ki >= 126) ? 0.f : __int_as_float((127 - ki) << 23);
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kLaunchBoundThreads, 1)
     sol_attn_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
                           const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_vb,
@@ -332,9 +391,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&ctl.s_full[b], 1);
-      mbar_init(&ctl.p_full[b], kSoftmaxThreads);
+      mbar_init(&ctl.p_full[b], kPFullCount);
+      mbar_init(&ctl.pv_done[b], 1);
+      mbar_init(&ctl.mready[b], 4);   // the four warps of the tile's warpgroup
     }
-    for (int b = 0; b < 3; ++b) mbar_init(&ctl.pv_done[b], 1);
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&ctl.ring_full[r], 1);
       mbar_init(&ctl.ring_empty[r], kRingEmptyCount);
@@ -345,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ctl.q_full, 1);
     mbar_init(&ctl.q_empty, 1);
-    mbar_init(&ctl.xchg, kSoftmaxThreads / 32);   // one arrival per softmax warp
+    mbar_init(&ctl.xchg, 8);   // one arrival per softmax warp
     ctl.abort = 0;
     fence_mbar_init();
   }
@@ -358,13 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl.tmem_base;
 
-  // Bounded wait; on a timeout raise the abort flag and the status word.  All
-  // later waits return false at once, every role leaves its loop, and the CTA
-  // meets at the final barrier.
   SA_PROF(unsigned long long prof[kPrSlots]; for (int i = 0; i < kPrSlots; ++i) prof[i] = 0;
           const unsigned long long prof_t0 = clock64();)
-  // The first probe is inline; the sleeping loop behind it is out of line,
-  // which keeps every wait site small.
+  // Bounded wait; on a timeout raise the abort flag and the status word.  All
+  // later waits return false at once, every role leaves its loop, and the CTA
+  // meets at the final barrier.  The first probe is inline; the sleeping loop
+  // behind it is out of line, which keeps every wait site small.
   auto wait = [&](uint64_t* bar, uint32_t parity, int slot) -> bool {
     SA_PROF(const unsigned long long tw = clock64();)
     const bool okw = mbar_try_wait(bar, parity) || wait_slow(bar, parity, abort_flag, p.status, p.timeout_ns);
@@ -376,10 +435,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto ring_get = [&](uint32_t r, int slot) -> bool {
     return wait(&ctl.ring_full[r % kRing], (r / kRing) & 1, slot);
   };
+  // A descriptor that points outside the head's blocks or items is a bug in
+  // the walk: record it, stop every role, never issue the copy.
+  auto bad_desc = [&]() {
+    *abort_flag = 1;
+    atomicOr(p.status, kStatusDevice);
+  };
 
-  if (warp == 10) {
+  if (warp >= 8 && warp < 12) {
+  if (warp == kWarpRoute) {
     // =========================================================== routing
-    for (int seq = 0;; ++seq) {
+    // (kFlagTestStall: publish nothing, so that every other role's bounded
+    // wait runs out; used only to exercise the timeout path.)
+    for (int seq = 0; !(p.flags & kFlagTestStall); ++seq) {
       const int s = seq & 1;
       if (seq >= 2 && !wait(&ctl.item_empty[s], ((seq >> 1) - 1) & 1, kPrRouteWait)) break;
       int item = 0;
@@ -454,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.item_full[s]);   // release: masks and item visible
     }
-  } else if (warp == 11) {
+  } else if (warp == kWarpSched) {
     // =========================================================== scheduler
     uint32_t r = 0;   // descriptors published
     const int NW = (p.N + 31) >> 5;
@@ -535,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.item_empty[s]);   // the item's masks are no longer read
     }
-  } else if (warp == 8) {
+  } else if (warp == kWarpLoad) {
     // =========================================================== TMA producers
     const bool kside = (lane == 0);
     if (lane < 2) {
@@ -549,6 +617,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&ctl.ring_empty[r % kRing]);
         if (flags & kDescEnd) break;
         if (flags & kDescEmpty) continue;
+        // range check of the coordinates this tile's copies use
+        if (bh < 0 || bh >= p.BH || pair < 0 || pair >= p.num_pairs || ja < 0 || ja >= p.N || jb >= p.N ||
+            ((flags & kDescApprox) && jb != -1)) {
+          bad_desc();
+          break;
+        }
         if (kside && (flags & kDescFirst)) {  // the item's query tile (the previous item's S MMAs must be done)
           if (qseq > 0 && !wait(&ctl.q_empty, (qseq - 1) & 1, kPrKQEmpty)) break;
           mbar_arrive_expect_tx(&ctl.q_full, 128u * D * 2u);
@@ -592,86 +666,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++stage == kStages) stage = 0;
       }
     }
-  } else if (warp == 9) {
-    // =========================================================== MMA issuer
-    // S(t) goes into TMEM buffer t % 3 and runs up to two tiles ahead of the
-    // PVs: for tile t this thread issues PV(t-2), then S(t) once PV(t-3), the
-    // last reader of the buffer, has completed.  PV(t-2) and S(t-1) sit
-    // between the two in the tensor pipe, so that wait rarely stalls it.
+  } else {
+    // =========================================================== S issuer
+    // S(t) = Q · Kside(t)ᵀ into TMEM buffer t % 3, once PV(t - 3), the last
+    // reader of that buffer, has completed.
     if (lane == 0) {
-      const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
+      const uint32_t sKa = smem_u32(sK);
       const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
-      int kstage = 0, vstage = 0;
-      uint32_t kphase = 0, vphase = 0;
-      uint32_t tcount = 0;           // tiles whose S MMA is issued
-      uint32_t qseq = 0;             // items with tiles seen
-      struct PendingPv {
-        uint32_t t, vphase;
-        int ncols, vstage;
-        bool first;
-      };
-      PendingPv pend[2];
-      int npend = 0;
-      bool ok = true;
-      // O (+)= P(t) · Vside(t), P read from TMEM buffer t % 3.  Softmax warpgroup
-      // w wrote the P of the tile's columns [w h, (w + 1) h), h = ncols / 2 (all
-      // 32 columns of a 32-column tile: warpgroup 0), as bf16 pairs starting at
-      // the buffer's column w h.
-      auto issue_pv = [&](const PendingPv& pv) -> bool {
-        const uint32_t b = pv.t % 3u;
-        if (!wait(&ctl.p_full[b], (pv.t / 3u) & 1u, kPrMmaP)) return false;
-        if (!wait(&ctl.v_full[pv.vstage], pv.vphase, kPrMmaV)) return false;
-        tc_fence_after();
-        SA_PROF(const unsigned long long tis = clock64();)
-        // descriptors are linear in the address: + (bytes >> 4) moves them
-        const uint64_t vdesc = sdesc_sw128(sVa + pv.vstage * kTile, CB, 1024);
-        const uint32_t pbase = tmem + kTmemS0 + 128u * b;
-        const uint32_t acc0 = pv.first ? 0u : 1u;
-        // K-step kk (keys 16 kk ..): P column 8 kk, + ncols / 4 for the second
-        // warpgroup's keys (a 32-column tile has only the first's)
-        if (pv.ncols == 128) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tmem + kTmemO, pbase + 8 * kk + (kk >= 4 ? 32 : 0), vdesc + 128 * kk, idesc_pv,
-                    kk == 0 ? acc0 : 1u);
-        } else if (pv.ncols == 64) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_ts(tmem + kTmemO, pbase + 8 * kk + (kk >= 2 ? 16 : 0), vdesc + 128 * kk, idesc_pv,
-                    kk == 0 ? acc0 : 1u);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            umma_ts(tmem + kTmemO, pbase + 8 * kk, vdesc + 128 * kk, idesc_pv, kk == 0 ? acc0 : 1u);
-        }
-        umma_commit(&ctl.pv_done[b]);
-        SA_PROF(prof[kPrMmaIssuePV] += clock64() - tis;)
-        return true;
-      };
-      auto pop_pv = [&]() -> bool {
-        const bool r = issue_pv(pend[0]);
-        pend[0] = pend[1];
-        --npend;
-        return r;
-      };
+      int kstage = 0;
+      uint32_t kphase = 0, tcount = 0, qseq = 0;
       for (uint32_t r = 0;; ++r) {
-        if (!ring_get(r, kPrMmaDesc)) { ok = false; break; }
+        if (!ring_get(r, kPrSDesc)) break;
         const TileDesc& dsc = ctl.ring[r % kRing];
         const int flags = dsc.flags, ncols = dsc.ncols;
         mbar_arrive(&ctl.ring_empty[r % kRing]);
         if (flags & kDescEnd) break;
         if (flags & kDescEmpty) continue;
-        if (npend == 2 && !pop_pv()) { ok = false; break; }   // PV(t-2)
-        const uint32_t b = tcount % 3u;
-        if (tcount >= 3 && !wait(&ctl.pv_done[b], ((tcount / 3u) - 1u) & 1u, kPrMmaSEmpty)) { ok = false; break; }
-        if (flags & kDescFirst) {
-          if (!wait(&ctl.q_full, qseq & 1, kPrMmaQ)) { ok = false; break; }
-        }
-        if (!wait(&ctl.k_full[kstage], kphase, kPrMmaK)) { ok = false; break; }
+        const uint32_t t = tcount++;
+        const uint32_t b = t % 3u;
+        if (t >= 3 && !wait(&ctl.pv_done[b], ((t / 3u) - 1u) & 1u, kPrSBuf)) break;
+        if ((flags & kDescFirst) && !wait(&ctl.q_full, qseq & 1, kPrSQ)) break;
+        if (!wait(&ctl.k_full[kstage], kphase, kPrSK)) break;
         tc_fence_after();
         SA_PROF(const unsigned long long tis = clock64();)
-        // S(t) = Q · Kside^T into buffer t % 3
         const uint32_t dS = tmem + kTmemS0 + 128u * b;
         const uint64_t kdesc = sdesc_sw128(sKa + kstage * kTile, 16, 1024);
         const uint32_t idesc_s = idesc_bf16_f32(128, ncols, 0);
@@ -688,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         umma_commit(&ctl.s_full[b]);
-        SA_PROF(prof[kPrMmaIssueS] += clock64() - tis;)
+        SA_PROF(prof[kPrSIssue] += clock64() - tis;)
         if (++kstage == kStages) {
           kstage = 0;
           kphase ^= 1u;
@@ -697,43 +714,80 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&ctl.q_empty);
           ++qseq;
         }
-        pend[npend++] = PendingPv{tcount, vphase, ncols, vstage, (flags & kDescFirst) != 0};
+      }
+    }
+  }
+  } else if (warp >= 12) {
+  if (warp == kWarpPv) {
+    // =========================================================== PV issuer
+    // O (+)= P(t) · Vside(t) in tile order, P read from TMEM buffer t % 3: the
+    // P of the tile's 16 kk .. 16 kk + 15 keys sits in the buffer's columns
+    // 8 kk .. 8 kk + 7 (bf16 pairs).
+    if (lane == 0) {
+      const uint32_t sVa = smem_u32(sV);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 1);
+      int vstage = 0;
+      uint32_t vphase = 0, tcount = 0;
+      for (uint32_t r = 0;; ++r) {
+        if (!ring_get(r, kPrPvDesc)) break;
+        const TileDesc& dsc = ctl.ring[r % kRing];
+        const int flags = dsc.flags, ncols = dsc.ncols;
+        mbar_arrive(&ctl.ring_empty[r % kRing]);
+        if (flags & kDescEnd) break;
+        if (flags & kDescEmpty) continue;
+        const uint32_t t = tcount++;
+        const uint32_t b = t % 3u;
+        if (!wait(&ctl.p_full[b], (t / 3u) & 1u, kPrPvP)) break;
+        if (!wait(&ctl.v_full[vstage], vphase, kPrPvV)) break;
+        tc_fence_after();
+        SA_PROF(const unsigned long long tis = clock64();)
+        // descriptors are linear in the address: + (bytes >> 4) moves them
+        const uint64_t vdesc = sdesc_sw128(sVa + vstage * kTile, CB, 1024);
+        const uint32_t pbase = tmem + kTmemS0 + 128u * b;
+        const uint32_t acc0 = (flags & kDescFirst) ? 0u : 1u;
+        if (ncols == 128) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tmem + kTmemO, pbase + 8 * kk, vdesc + 128 * kk, idesc_pv, kk == 0 ? acc0 : 1u);
+        } else if (ncols == 64) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tmem + kTmemO, pbase + 8 * kk, vdesc + 128 * kk, idesc_pv, kk == 0 ? acc0 : 1u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            umma_ts(tmem + kTmemO, pbase + 8 * kk, vdesc + 128 * kk, idesc_pv, kk == 0 ? acc0 : 1u);
+        }
+        umma_commit(&ctl.pv_done[b]);
+        SA_PROF(prof[kPrPvIssue] += clock64() - tis;)
         if (++vstage == kStages) {
           vstage = 0;
           vphase ^= 1u;
         }
-        ++tcount;
       }
-      while (ok && npend > 0) ok = pop_pv();
     }
+  }
   } else {
     // =========================================================== softmax (warps 0-7)
-    // Both warpgroups work on every tile: the thread of warpgroup wg and TMEM
-    // lane `row` owns tile row `row` and the tile's columns [wg h, (wg + 1) h),
-    // h = ncols / 2 (a 32-column tile belongs to warpgroup 0 alone).  The two
-    // threads of a row share one reference maximum m (log2 units) and keep
-    // partial row sums l; P of the tile accumulates into the single O.
+    // Tile t belongs to warpgroup t & 1; the thread of TMEM lane `row` owns row
+    // `row` of it, every column.  m and the row sums are in log2 units.
     const int wg = warp >> 2;
     const int row = tid & 127;        // tile row = TMEM lane
     const int half = row >> 6;        // query block of the pair the row belongs to
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tmem + kTmemO + lane_base;
-    uint32_t tcount = 0;     // tiles processed (S buffer tcount % 3, PV index tcount)
-    uint32_t xc = 0;         // exchanges done
-    // Exchange one value per row with the other warpgroup's thread of the row.
-    auto exchange = [&](float a) -> float {
-      const int ph = xc & 1;
-      ctl.xval[ph][wg][row] = a;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.xchg);
-      wait(&ctl.xchg, ph, kPrSmX);
-      ++xc;
-      return ctl.xval[ph][wg ^ 1][row];
+    uint32_t tcount = 0;     // tiles seen (S buffer tcount % 3, PV index tcount)
+    uint32_t xc = 0;         // epilogue exchanges done
+    float l_run = 0.f;       // this thread's partial row sum ...
+    float m_l = -INFINITY;   // ... accumulated at this reference maximum
+    float m_own = -INFINITY; // the m this warpgroup's latest tile of the item settled on
+    bool item_tiles = false; // the current item had a tile
+    // The warp leaves together: its TMEM loads and stores are warp-wide.
+    auto wait_w = [&](uint64_t* bar, uint32_t parity, int slot) -> bool {
+      return __all_sync(0xFFFFFFFFu, wait(bar, parity, slot));
     };
-    float m_run = -INFINITY, l_run = 0.f;
-    bool item_tiles = false;  // the current item had a tile
     for (uint32_t r = 0;; ++r) {
-      if (!ring_get(r, kPrSmDesc)) break;
+      if (!wait_w(&ctl.ring_full[r % kRing], (r / kRing) & 1, kPrSmDesc)) break;
       const TileDesc& dsc = ctl.ring[r % kRing];
       const uint4 bw = *reinterpret_cast<const uint4*>(dsc.bits[half]);
       const int ncols = dsc.ncols, dflags = dsc.flags, tail_col = dsc.tail, dbh = dsc.bh, dpair = dsc.pair;
@@ -743,153 +797,169 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(dflags & kDescEmpty)) {
         const uint32_t t = tcount++;
         const uint32_t b = t % 3u;
-        wait(&ctl.s_full[b], (t / 3u) & 1u, kPrSmS);
-        tc_fence_after();
-        SA_PROF(unsigned long long tph = clock64(); prof[kPrSmTiles] += 1;)
         const bool first = (dflags & kDescFirst) != 0;
         if (first) {
-          m_run = -INFINITY;
           l_run = 0.f;
+          m_l = -INFINITY;
+          m_own = -INFINITY;
         }
         item_tiles = true;
-        const int hw = (ncols == 32) ? (wg == 0 ? 32 : 0) : (ncols >> 1);   // this thread's columns
-        const int c0 = (ncols == 32) ? 0 : wg * hw;                           // their first column
-        const int ng = hw >> 5;                                               // 32-column groups: 0, 1, 2
-        const uint32_t tS = tmem + kTmemS0 + 128u * b + lane_base;
-        auto gb = [&](int i) -> uint32_t { return i == 0 ? bw.x : i == 1 ? bw.y : i == 2 ? bw.z : bw.w; };
-        // Column adjustments, only where needed: invalid columns become -inf,
-        // the ragged block's approximation column gets log2(n_tail / 64).
-        const int tail_g = tail_col >= 0 ? (tail_col >> 5) : -1;
-        auto adjust = [&](float* xv, int g) {
-          const uint32_t bits = gb(g);
-          const int et = (g == tail_g) ? (tail_col & 31) : -1;
-          if (bits != 0xFFFFFFFFu || et >= 0) {
+        if (static_cast<int>(t & 1u) != wg) {
+          // Not this warpgroup's tile.  On an item's first tile both warpgroups
+          // arrive, so that its PV (which overwrites O) waits for this
+          // warpgroup's epilogue reads of the previous item's O.
+          if (first) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cnt(&ctl.p_full[b], 1u);
+          }
+        } else {
+          if (!wait_w(&ctl.s_full[b], (t / 3u) & 1u, kPrSmS)) break;
+          tc_fence_after();
+          SA_PROF(unsigned long long tph = clock64(); prof[kPrSmTiles] += 1;)
+          const int ng = ncols >> 5;                 // 32-column groups: 1, 2 or 4
+          const uint32_t tS = tmem + kTmemS0 + 128u * b + lane_base;
+          auto gb = [&](int i) -> uint32_t { return i == 0 ? bw.x : i == 1 ? bw.y : i == 2 ? bw.z : bw.w; };
+          // Column adjustments, only where needed: invalid columns become -inf,
+          // the ragged block's approximation column gets log2(n_tail / 64).
+          const int tail_g = tail_col >= 0 ? (tail_col >> 5) : -1;
+          auto adjust = [&](float* xv, int g) {
+            const uint32_t bits = gb(g);
+            const int et = (g == tail_g) ? (tail_col & 31) : -1;
+            if (bits != 0xFFFFFFFFu || et >= 0) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (e == et) xv[e] += p.tail_raw;
-              if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
+              for (int e = 0; e < 32; ++e) {
+                if (e == et) xv[e] += p.tail_raw;
+                if (!((bits >> e) & 1u)) xv[e] = -INFINITY;
+              }
             }
-          }
-        };
-        // In log2 units.  An approximation column stands for its n_j tokens:
-        // its weight n_j is folded into the logit as + log2(n_j) (6 for a full
-        // block) and the value side uses the block mean V̂_j / n_j.
-        const float boost = (dflags & kDescApprox) ? 6.f : 0.f;
-        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-        // p = 2^y, y = x * scale_log2 + off, for 32 adjusted columns, packed as
-        // 16 bf16 pairs; the fp32 values go into the row sum (ra, rb) and the
-        // largest y into ym.
-        auto probs32 = [&](const float* xv, float2 of2, uint32_t* pk, float2& ra, float2& rb, float& ym) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
-            const float2 y1 = __ffma2_rn(make_float2(xv[e + 2], xv[e + 3]), sc2, of2);
-            const float2 y2 = __ffma2_rn(make_float2(xv[e + 4], xv[e + 5]), sc2, of2);
-            const float2 y3 = __ffma2_rn(make_float2(xv[e + 6], xv[e + 7]), sc2, of2);
-            ym = max3f(ym, max3f(y0.x, y0.y, y1.x), max3f(y1.y, y2.x, y2.y));
-            ym = max3f(ym, y3.x, y3.y);
-            const float2 q0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
-            const float2 q1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
-            const float2 q2 = make_float2(ex2_approx(y2.x), ex2_approx(y2.y));
-            const float2 q3 = make_float2(ex2_approx(y3.x), ex2_approx(y3.y));
-            ra = __fadd2_rn(ra, __fadd2_rn(q0, q2));
-            rb = __fadd2_rn(rb, __fadd2_rn(q1, q3));
-            pk[e >> 1] = pack_bf16x2(q0.x, q0.y);
-            pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
-            pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
-            pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
-          }
-        };
-        // This thread's columns, against the reference maximum mref: P into
-        // pk[0, 16 ng), the row sum into (ra, rb); returns the largest y.
-        auto own_cols = [&](float mref, uint32_t* pk, float2& ra, float2& rb) -> float {
-          const float2 of2 = make_float2(boost - mref, boost - mref);
-          float ym = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            if (i < ng) {
-              float xv[32];
-              tmem_ld_x32f(tS + c0 + 32 * i, xv);
-              tmem_ld_wait();
-              reg_fence32(xv);
-              adjust(xv, (c0 >> 5) + i);
-              probs32(xv, of2, pk + 16 * i, ra, rb, ym);
-            }
-          }
-          return ym;
-        };
-        // One pass against the row's reference maximum m (0 while the row has
-        // seen no valid column), P held in registers.  Each thread proposes the
-        // m it needs: m itself while its y stay <= 8 (the lazy rescale rule),
-        // else m raised by a whole number k of doublings (so that everything
-        // accumulated so far scales by 2^-k exactly, even P already in bf16),
-        // or its maximum rounded up on the row's first valid column.  The two
-        // threads of the row agree on the larger proposal; where it moved, l
-        // and this thread's half of O scale by 2^(m - m') and the columns are
-        // recomputed from S, which no P store has reached yet.
-        uint32_t pk[32];
-        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-        const float ym = own_cols(m_run == -INFINITY ? 0.f : m_run, pk, sa, sb);
-        // m stays a whole number (its first value is rounded up), so that every
-        // later step m' - m is exact in fp32
-        const float prop = (m_run == -INFINITY) ? ceilf(ym) : (ym > 8.f ? m_run + ceilf(ym) : m_run);
-        const float m_new = fmaxf(prop, exchange(prop));
-        const bool moved = !(m_new == m_run);
-        if (__any_sync(0xFFFFFFFFu, moved)) {
-          SA_PROF(prof[kPrSmRedo] += 1;)
-          float alpha = 1.f;
-          if (moved) {
-            if (m_run == -INFINITY) {
-              alpha = 0.f;   // nothing valid accumulated yet
-            } else {
-              const int k = __float2int_rn(m_new - m_run);
-              alpha = (k >= 126) ? 0.f : __int_as_float((127 - k) << 23);
-            }
-            l_run *= alpha;
-            m_run = m_new;
-          }
-          __syncwarp();
-          if (!first) {
-            // O holds PV(0 .. t-1) of the item; wait for PV(t-1), then scale this
-            // thread's half of the row
-            wait(&ctl.pv_done[(t - 1u) % 3u], ((t - 1u) / 3u) & 1u, kPrSmO);
-            tc_fence_after();
+          };
+          // One pass over the row's columns, 32 at a time, against a running
+          // reference m_cur that starts at the m this warpgroup's previous tile
+          // of the item settled on.  A group whose largest y exceeds m_cur by
+          // more than 8 raises m_cur to a whole number (the groups already
+          // stored are scaled by the exact power of two).  Afterwards m_cur
+          // meets the m that tile t - 1 settled on; the larger wins, and P or
+          // O, whichever is behind, is scaled to it (both are rare).
+          const float boost = (dflags & kDescApprox) ? 6.f : 0.f;
+          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+          float m_cur = m_own;
+          float2 ra = make_float2(0.f, 0.f), rb = make_float2(0.f, 0.f);
 #pragma unroll 1
-            for (int c16 = wg * (D / 2); c16 < (wg + 1) * (D / 2); c16 += 16) {
-              float rr[16];
-              tmem_ld_x16f(tO + c16, rr);
-              tmem_ld_wait();
-              reg_fence16(rr);
-              uint32_t pw[16];
+          for (int g = 0; g < ng; ++g) {
+            float xv[32];
+            SA_PROF(const unsigned long long tl0 = clock64();)
+            tmem_ld_x32f(tS + 32 * g, xv);
+            tmem_ld_wait();
+            reg_fence32(xv);
+            SA_PROF(prof[kPrSmLd] += clock64() - tl0;)
+            adjust(xv, g);
+            const float ym = max32(xv) * p.scale_log2 + boost;   // -inf: no valid column here
+            const bool up = ym > m_cur + 8.f;
+            if (__any_sync(0xFFFFFFFFu, up)) {
+              const float m_new = up ? ceilf(ym) : m_cur;
+              const float f = (m_cur == -INFINITY) ? 0.f : exp2_neg_int(m_new - m_cur);
+              scale_p(tS, g, f);
+              ra.x *= f; ra.y *= f; rb.x *= f; rb.y *= f;
+              m_cur = m_new;
+            }
+            const float mref = (m_cur == -INFINITY) ? 0.f : m_cur;
+            const float2 of2 = make_float2(boost - mref, boost - mref);
+            SA_PROF(const unsigned long long te0 = clock64();)
+            uint32_t pk[16];
 #pragma unroll
-              for (int e = 0; e < 16; ++e) pw[e] = __float_as_uint(rr[e] * alpha);
-              tmem_st_x16(tO + c16, pw);
+            for (int e = 0; e < 32; e += 8) {
+              const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
+              const float2 y1 = __ffma2_rn(make_float2(xv[e + 2], xv[e + 3]), sc2, of2);
+              const float2 y2 = __ffma2_rn(make_float2(xv[e + 4], xv[e + 5]), sc2, of2);
+              const float2 y3 = __ffma2_rn(make_float2(xv[e + 6], xv[e + 7]), sc2, of2);
+              const float2 q0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+              const float2 q1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+              const float2 q2 = make_float2(ex2_approx(y2.x), ex2_approx(y2.y));
+              const float2 q3 = make_float2(ex2_approx(y3.x), ex2_approx(y3.y));
+              ra = __fadd2_rn(ra, __fadd2_rn(q0, q2));
+              rb = __fadd2_rn(rb, __fadd2_rn(q1, q3));
+              pk[e >> 1] = pack_bf16x2(q0.x, q0.y);
+              pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
+              pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
+              pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
+            }
+            tmem_st_x16(tS + 16 * g, pk);
+            SA_PROF(prof[kPrSmExp] += clock64() - te0;)
+          }
+          SA_PROF(prof[kPrSmPass] += clock64() - tph; tph = clock64();)
+          // ---- meet the m of tile t - 1 (its owner published it at its end)
+          float m_hand = -INFINITY;
+          if (!first) {
+            const uint32_t tp = t - 1u;
+            if (!wait_w(&ctl.mready[tp % 3u], (tp / 3u) & 1u, kPrSmHand)) break;
+            m_hand = ctl.hand[tp % 3u][row];
+          }
+          const float m_fin = fmaxf(m_cur, m_hand);
+          const bool p_behind = (m_fin != m_cur) && (m_cur != -INFINITY);
+          if (__any_sync(0xFFFFFFFFu, p_behind)) {   // tile t - 1 raised m: scale this tile's P
+            const float f = p_behind ? exp2_neg_int(m_fin - m_cur) : 1.f;
+            scale_p(tS, ng, f);
+            ra.x *= f; ra.y *= f; rb.x *= f; rb.y *= f;
+          }
+          const bool o_behind = (m_fin != m_hand) && (m_hand != -INFINITY);
+          if (__any_sync(0xFFFFFFFFu, o_behind)) {   // this tile raised m: scale O (PV(0 .. t - 1))
+            if (!wait_w(&ctl.pv_done[(t - 1u) % 3u], ((t - 1u) / 3u) & 1u, kPrSmO)) break;
+            tc_fence_after();
+            const float alpha = o_behind ? exp2_neg_int(m_fin - m_hand) : 1.f;
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+              float o[32];
+              tmem_ld_x32f(tO + c, o);
+              tmem_ld_wait();
+              reg_fence32(o);
+              uint32_t ow[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ow[e] = __float_as_uint(o[e] * alpha);
+              tmem_st_x32(tO + c, ow);
             }
             SA_PROF(prof[kPrSmRescales] += 1;)
           }
-          sa = make_float2(0.f, 0.f);
-          sb = make_float2(0.f, 0.f);
-          (void)own_cols(m_run == -INFINITY ? 0.f : m_run, pk, sa, sb);
+          ctl.hand[b][row] = m_fin;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.mready[b]);
+          m_own = m_fin;
+          // this thread's partial row sum follows the reference
+          const float tile_sum = (ra.x + ra.y) + (rb.x + rb.y);
+          l_run = (m_l == -INFINITY || m_l == m_fin) ? l_run : l_run * exp2_neg_int(m_fin - m_l);
+          l_run += tile_sum;
+          m_l = m_fin;
+          tmem_st_wait();
+          SA_PROF(prof[kPrSmMeet] += clock64() - tph;)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cnt(&ctl.p_full[b], first ? 1u : 2u);
         }
-        // P of this thread's columns lands in TMEM columns [c0, c0 + hw / 2),
-        // inside its own part of S, which it has read
-        if (ng > 0) tmem_st_x16(tS + c0, pk);
-        if (ng > 1) tmem_st_x16(tS + c0 + 16, pk + 16);
-        l_run += (sa.x + sa.y) + (sb.x + sb.y);
-        tmem_st_wait();
-        SA_PROF(prof[kPrSmPass2] += clock64() - tph;)
-        tc_fence_before();
-        mbar_arrive(&ctl.p_full[b]);
       }
       if (!(dflags & (kDescLast | kDescEmpty))) continue;
-      // ---- epilogue: O / (l_0 + l_1) for this thread's half of the row's columns
+      // ---- epilogue: O / (l_0 + l_1) for this warpgroup's half of the row's columns
       SA_PROF(const unsigned long long tep = clock64();)
       if (item_tiles) {   // the item's last PV
-        wait(&ctl.pv_done[(tcount - 1u) % 3u], ((tcount - 1u) / 3u) & 1u, kPrSmO);
+        if (!wait_w(&ctl.pv_done[(tcount - 1u) % 3u], ((tcount - 1u) / 3u) & 1u, kPrSmO)) break;
         tc_fence_after();
       }
-      const float my_l = item_tiles ? l_run : 0.f;
-      const float l_tot = my_l + exchange(my_l);
+      const float2 mine = item_tiles ? make_float2(l_run, m_l) : make_float2(0.f, -INFINITY);
+      float2 other;
+      {
+        const int ph = xc & 1;
+        ctl.xval[ph][wg][row] = mine;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.xchg);
+        if (!wait_w(&ctl.xchg, ph, kPrSmX)) break;
+        ++xc;
+        other = ctl.xval[ph][wg ^ 1][row];
+      }
+      // O was accumulated at the item's last reference maximum, the larger of
+      // the two partials' (m never falls)
+      const float m_f = fmaxf(mine.y, other.y);
+      float l_tot = 0.f;
+      if (mine.y != -INFINITY) l_tot += mine.x * exp2_neg_int(m_f - mine.y);
+      if (other.y != -INFINITY) l_tot += other.x * exp2_neg_int(m_f - other.y);
       const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
       const int token = 128 * dpair + row;
       uint16_t* orow = p.out + (static_cast<size_t>(dbh) * p.L + token) * D;
@@ -913,7 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // O is read; the next item's first PV (which overwrites O) waits for this
-      // thread's next P arrival, which comes after these reads
+      // warp's arrival on that tile, which comes after these reads
       tc_fence_before();
       item_tiles = false;
       SA_PROF(prof[kPrSmEpi] += clock64() - tep;)
@@ -921,9 +991,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   SA_PROF({
-    const int tslot = warp == 10 ? kPrTotRoute : warp == 11 ? kPrTotSched : warp == 9 ? kPrTotMma
-                    : warp == 8 ? (lane == 0 ? kPrTotK : kPrTotV) : kPrTotSm;
-    if ((lane == 0 && (warp >= 8 || warp == 0)) || (warp == 8 && lane == 1)) {
+    const int tslot = warp == kWarpRoute ? kPrTotRoute : warp == kWarpSched ? kPrTotSched
+                    : warp == kWarpS ? kPrTotS : warp == kWarpPv ? kPrTotPv
+                    : warp == kWarpLoad ? (lane == 0 ? kPrTotK : kPrTotV) : kPrTotSm;
+    // one thread per role; the softmax slots come from the first warp of each
+    // warpgroup, so they cover every tile once
+    if ((lane == 0 && (warp >= 8 || warp == 0 || warp == 4)) || (warp == kWarpLoad && lane == 1)) {
       prof[tslot] = clock64() - prof_t0;
       for (int i = 0; i < kPrSlots; ++i) if (prof[i]) atomicAdd(&g_profile[i], prof[i]);
     }

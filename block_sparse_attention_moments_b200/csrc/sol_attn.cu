@@ -23,7 +23,9 @@ namespace {
 
 constexpr int kBlock = 64;
 constexpr int kMaxL = 1 << 20;
+constexpr int kMaxBH = 65535;
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // bounded device waits: 2 s
+constexpr unsigned long long kTestTimeoutNs = 1000000ull;  // with SOL_ATTN_FLAG_TEST_STALL: 1 ms
 
 thread_local std::string g_last_error;
 
@@ -171,7 +173,10 @@ int check_shape(int B, int H, int L, int d, int block) {
   if (block != kBlock) return fail(SOL_ATTN_ERR_UNSUPPORTED, "block must be 64 (got %d)", block);
   if (d != 64 && d != 128) return fail(SOL_ATTN_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
   if (L > kMaxL) return fail(SOL_ATTN_ERR_UNSUPPORTED, "L = %d exceeds the supported maximum %d", L, kMaxL);
-  if (static_cast<long long>(B) * H > (1LL << 24)) return fail(SOL_ATTN_ERR_UNSUPPORTED, "B*H too large");
+  // pool, moments and threshold kernels put B*H on gridDim.y (at most 65535)
+  if (static_cast<long long>(B) * H > kMaxBH)
+    return fail(SOL_ATTN_ERR_UNSUPPORTED, "B*H = %lld exceeds the supported maximum %d",
+                static_cast<long long>(B) * H, kMaxBH);
   return SOL_ATTN_OK;
 }
 
@@ -327,7 +332,9 @@ int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void
   p.out = static_cast<uint16_t*>(out);
   p.work_counter = w.counter;
   p.status = w.status;
-  p.timeout_ns = kTimeoutNs;
+  // SOL_ATTN_FLAG_TEST_STALL: the routing warp publishes nothing and every
+  // wait gives up after 1 ms (exercises the timeout path; no output is written)
+  p.timeout_ns = (flags & SOL_ATTN_FLAG_TEST_STALL) ? kTestTimeoutNs : kTimeoutNs;
 
   int dev = 0, nsm = 0;
   CUDA_TRY(cudaGetDevice(&dev));
@@ -363,7 +370,7 @@ int read_status(Workspace& w, cudaStream_t st) {
   if (h) {
     CUDA_TRY(cudaMemset(w.status, 0, sizeof(unsigned)));
     if (h & kStatusTimeout) return fail(SOL_ATTN_ERR_TIMEOUT, "a bounded device wait gave up (status 0x%x)", h);
-    return fail(SOL_ATTN_ERR_DEVICE, "device-side check failed (status 0x%x)", h);
+    return fail(SOL_ATTN_ERR_DEVICE, "device-side check failed: a tile descriptor was out of range (status 0x%x)", h);
   }
   return SOL_ATTN_OK;
 }

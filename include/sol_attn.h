@@ -21,7 +21,8 @@
  *     address 16-byte aligned.  out must not overlap q, k or v.
  *   - block must be 64 (fixed 64x64 physical blocks, experiments: setup);
  *     d must be 64 or 128; N = ceil(L / 64); the last block may be ragged and
- *     is pooled over its valid tokens.  1 <= L <= 1,048,576, chunk >= 1.
+ *     is pooled over its valid tokens.  1 <= L <= 1,048,576, chunk >= 1,
+ *     1 <= B*H <= 65535.
  *   - beta: any finite value; -INFINITY selects every block (dense mode),
  *     +INFINITY selects none (every block approximated); NaN is rejected.
  *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
@@ -48,12 +49,16 @@ extern "C" {
 typedef enum sol_attn_status {
   SOL_ATTN_OK = 0,
   SOL_ATTN_ERR_ARG = -1,          /* null pointer, non-positive size, NaN beta, chunk < 1 */
-  SOL_ATTN_ERR_UNSUPPORTED = -2,  /* d not in {64,128}, block != 64, L too large, not sm_100 */
+  SOL_ATTN_ERR_UNSUPPORTED = -2,  /* d not in {64,128}, block != 64, L too large, B*H > 65535,
+                                     not sm_100 */
   SOL_ATTN_ERR_ALIGN = -3,        /* a tensor base address is not 16-byte aligned */
   SOL_ATTN_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
   SOL_ATTN_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up (status word) */
   SOL_ATTN_ERR_STATE = -6,        /* stats/stage call without a matching earlier forward */
-  SOL_ATTN_ERR_DEVICE = -7        /* a device-side consistency check failed (status word) */
+  SOL_ATTN_ERR_DEVICE = -7        /* a device-side consistency check failed (status word):
+                                     the fused kernel range-checks every tile descriptor
+                                     (head, query pair, key blocks) before its copies and
+                                     stops instead of issuing an out-of-range one */
 } sol_attn_status;
 
 /* Flags for sol_attn_forward_ex. */
@@ -62,6 +67,11 @@ typedef enum sol_attn_status {
                                           blocks (ablation: exact-only vs exact-or-approx) */
 #define SOL_ATTN_FLAG_SYNC_CHECK 0x4u  /* synchronise the stream after the forward and read
                                           the device status word (timeouts, device checks) */
+#define SOL_ATTN_FLAG_TEST_STALL 0x8u  /* test of the failure path only: the fused kernel's
+                                          routing step publishes no work, every bounded wait
+                                          gives up after 1 ms, the kernel exits cleanly and
+                                          the status word reports SOL_ATTN_ERR_TIMEOUT; out
+                                          is left unwritten */
 
 /* Optional device buffers filled by sol_attn_forward_ex (any member may be NULL).
  * Shapes use N = ceil(L/64); all are row-major and owned by the caller. */
@@ -79,8 +89,8 @@ typedef struct sol_attn_debug {
 /* Sol-Attn forward (method: Eq. 3-11).  q, k, v: input [B,H,L,d] bf16 device
  * tensors; out: output [B,H,L,d] bf16 device tensor, every valid row written.
  * chunk: C, the number of pooled keys routed per outer-loop step (Eq. 6); it
- * changes the schedule, not the result.  Enqueues three kernels (pool,
- * moments, fused attention) on stream. */
+ * changes the schedule, not the result.  Enqueues a memset of the work counter
+ * and four kernels (pool, moments, thresholds, fused attention) on stream. */
 int sol_attn_forward(const void* q, const void* k, const void* v, void* out,
                      int B, int H, int L, int d, int block, int chunk, float beta,
                      void* stream);

@@ -229,3 +229,21 @@ def test_approximation_ablation_on_device(beta):
     print(f"beta={beta} rel-l2 vs select-all: approx {r_full:.2e} exact-only {r_exact:.2e}")
     assert r_full < 5e-3              # bf16 rounding of P and of the output only
     assert r_exact > 10 * max(r_full, 1e-4)
+
+
+def test_bounded_wait_runs_out_and_the_next_forward_is_clean():
+    # Failure path of the fused kernel's bounded waits: with the test-stall flag
+    # its routing step publishes no work, every waiting role gives up after
+    # 1 ms and leaves, TMEM is released and the status word says "timeout".
+    # The context stays usable: the next forward (status cleared) passes parity.
+    import torch
+    from parity_util import to_device
+    wl = WORKLOADS["tiny"]
+    qb, kb, vb = fourier_inputs(wl)
+    q, k, v = to_device(qb), to_device(kb), to_device(vb)
+    with pytest.raises(sa.SolAttnError) as e:
+        sa.forward(q, k, v, 1.0, wl.chunk, flags=sa.FLAG_TEST_STALL | sa.FLAG_SYNC_CHECK)
+    assert e.value.code == -5
+    assert "timed out" in str(e.value)
+    torch.cuda.synchronize()
+    _full_check(qb, kb, vb, 1.0, wl.chunk)
