@@ -41,6 +41,7 @@ EXPORTED_SYMBOLS = (
     "sol_attn_stage_pool", "sol_attn_stage_threshold", "sol_attn_stage_fused",
     "sol_attn_workspace_bytes", "sol_attn_release", "sol_attn_error_string",
     "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc", "sol_attn_profile_read",
+    "sol_attn_noalloc_status",
 )
 
 
@@ -85,9 +86,11 @@ def lib():
     L.sol_attn_kernels_per_forward.argtypes = []
     L.sol_attn_forward_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.sol_attn_profile_read.argtypes = [vp, i, i]
+    L.sol_attn_noalloc_status.argtypes = [vp]
     for name in ("sol_attn_forward", "sol_attn_forward_ex", "sol_attn_stats", "sol_attn_forward_host",
                  "sol_attn_stage_pool", "sol_attn_stage_threshold", "sol_attn_stage_fused", "sol_attn_release",
-                 "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc", "sol_attn_profile_read"):
+                 "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc", "sol_attn_profile_read",
+                 "sol_attn_noalloc_status"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L

@@ -676,9 +676,32 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
   layout(s, &w, static_cast<char*>(w.base));
   w.shape = s;
   auto st = static_cast<cudaStream_t>(stream);
+  // the status word reports on this call only (read by sol_attn_noalloc_status)
+  CUDA_TRY(cudaMemsetAsync(w.status, 0, sizeof(unsigned), st));
   if ((rc = run_pool(w, q, k, v, nullptr, st))) return rc;
   if ((rc = run_threshold(w, beta, 0u, nullptr, st))) return rc;
   return run_fused(w, q, k, v, out, chunk, 0u, nullptr, st);
+}
+
+int sol_attn_noalloc_status(void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  if (!g_noalloc_base[dev])
+    return fail(SOL_ATTN_ERR_STATE, "no allocation-free forward has run on device %d", dev);
+  auto st = static_cast<cudaStream_t>(stream);
+  unsigned* status = reinterpret_cast<unsigned*>(g_noalloc_base[dev]) + 32;
+  unsigned h = 0;
+  CUDA_TRY(cudaMemcpyAsync(&h, status, sizeof(h), cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  if (h) {
+    CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(unsigned), st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    if (h & kStatusTimeout) return fail(SOL_ATTN_ERR_TIMEOUT, "a bounded device wait gave up (status 0x%x)", h);
+    return fail(SOL_ATTN_ERR_DEVICE, "device-side check failed: a tile descriptor was out of range (status 0x%x)",
+                h);
+  }
+  return SOL_ATTN_OK;
 }
 
 }  // extern "C"

@@ -164,10 +164,20 @@ int sol_attn_profile_read(uint64_t* cycles, int n, int reset);
  * outside any stream capture.  All calls on a device share the array and it
  * keeps the last call's contents: calls that overlap on the GPU (different
  * streams, or host threads racing) race on it and must be serialised by the
- * caller.  sol_attn_stats does not report on these calls. */
+ * caller.  sol_attn_stats does not report on these calls; sol_attn_noalloc_status
+ * reads the call's device status word. */
 int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out,
                              int B, int H, int L, int d, int block, int chunk, float beta,
                              void* stream);
+
+/* Status of the last allocation-free forward on this device (the paper has no
+ * counterpart).  That forward clears the device status word when it is
+ * enqueued; this call synchronises stream, copies the word to the host (no
+ * allocation), clears it and returns SOL_ATTN_OK, SOL_ATTN_ERR_TIMEOUT (a
+ * bounded wait of the fused kernel gave up; out is not valid) or
+ * SOL_ATTN_ERR_DEVICE.  SOL_ATTN_ERR_STATE if no allocation-free forward has
+ * run on this device.  Pass the stream the forward was enqueued on. */
+int sol_attn_noalloc_status(void* stream);
 
 #ifdef __cplusplus
 }

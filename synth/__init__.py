@@ -35,7 +35,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "WORKLOADS", "grid_coords", "fourier_inputs", "gauss_inputs", "ramp_inputs", "offset_inputs",
-    "bf16_round", "bf16_bits_to_f64", "f32_to_bf16_bits", "f32_to_bf16_bits_np",
+    "near_block_constant_keys", "bf16_round", "bf16_bits_to_f64", "f32_to_bf16_bits", "f32_to_bf16_bits_np",
 ]
 
 
@@ -198,3 +198,18 @@ def custom_fourier(B: int, H: int, grid, d: int, amp: float, seed: int):
     """Fourier-feature inputs for an arbitrary grid (edge-case shapes in tests)."""
     wl = Workload("custom", B, H, tuple(grid), d, 1, (1.0,), amp, seed)
     return fourier_inputs(wl)
+
+
+def near_block_constant_keys(kb: np.ndarray, eps: float, seed: int, block: int = 64) -> np.ndarray:
+    """bf16 key bits [B, H, L, d] in which every key of a 64-token block is the
+    block's first key of ``kb`` plus eps * N(0, 1) noise: keys nearly constant
+    within a block, the regime in which the approximation of unselected blocks
+    carries a large share of each row's softmax mass."""
+    k = bf16_bits_to_f64(kb).astype(np.float32)
+    L = k.shape[2]
+    for j in range(0, L, block):
+        k[:, :, j:j + block, :] = k[:, :, j:j + 1, :]
+    rng = np.random.default_rng(seed)
+    k = k + np.float32(eps) * rng.standard_normal(size=k.shape, dtype=np.float32)
+    return f32_to_bf16_bits(k)
+

@@ -3,18 +3,28 @@ and compare it with the fp64 oracle on the same seeded bf16 inputs.
 
 Tolerances (the workload statement): selection masks bit-exact except for
 blocks whose proxy logit lies within 1e-4 of the row threshold (counted and
-reported); outputs within max-abs 2e-2 and relative-l2 5e-3.
+reported); outputs within max-abs 2e-2 and relative-l2 5e-3, for every
+(batch, head) slice on its own.
 """
 import math
 
 import numpy as np
 
-from oracle import proxy_row, sol_attn_head
+from oracle import (key_moments, pool_blocks, proxy_logits, proxy_row, row_stats_from_moments,
+                    select_global, sol_attn_head, thresholds)
 from synth import bf16_bits_to_f64
 
 BAND = 1e-4
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
+# A disagreement between the GPU's and the oracle's selection is only allowed
+# inside the band; their number must also stay a tiny fraction of the entries
+# compared (the band is narrow next to the spread of the proxy logits).
+MAX_BAND_FRACTION = 1e-4
+
+# Band statistics of the whole session, printed by conftest.py at the end of
+# the run: entries compared, entries inside the band, disagreements.
+SESSION = {"mask_entries": 0, "in_band": 0, "band_mismatch": 0, "count_rows": 0}
 
 
 def to_device(bits):
@@ -37,32 +47,103 @@ def run_gpu(qb, kb, vb, beta, chunk, flags=0, debug=True):
 
 
 class Report:
+    """Output errors per (batch, head) slice and mask agreement of one test."""
+
     def __init__(self):
+        self.heads = {}           # (b, h) -> [max_abs, sum sq err, sum sq ref, rows]
+        self.mask_entries = 0
+        self.in_band = 0
         self.band_mismatch = 0
-        self.rows = 0
-        self.max_abs = 0.0
-        self.num = 0.0
-        self.den = 0.0
+
+    def add_rows(self, b, h, g, r):
+        e = self.heads.setdefault((b, h), [0.0, 0.0, 0.0, 0])
+        e[0] = max(e[0], float(np.abs(g - r).max()))
+        e[1] += float(((g - r) ** 2).sum())
+        e[2] += float((r ** 2).sum())
+        e[3] += 1
+
+    def per_head(self):
+        return {k: (v[0], math.sqrt(v[1] / v[2]) if v[2] > 0 else 0.0, v[3]) for k, v in self.heads.items()}
+
+    @property
+    def max_abs(self):
+        return max((v[0] for v in self.per_head().values()), default=0.0)
 
     @property
     def rel_l2(self):
-        return math.sqrt(self.num / self.den) if self.den > 0 else 0.0
+        """Worst per-head relative l2 error."""
+        return max((v[1] for v in self.per_head().values()), default=0.0)
 
     def check(self):
-        assert self.max_abs <= MAX_ABS, f"max-abs {self.max_abs:.3e} > {MAX_ABS}"
-        assert self.rel_l2 <= REL_L2, f"rel-l2 {self.rel_l2:.3e} > {REL_L2}"
+        bad = {k: v for k, v in self.per_head().items() if v[0] > MAX_ABS or v[1] > REL_L2}
+        assert not bad, f"heads over tolerance (max-abs, rel-l2, rows): {bad}; {self}"
+        assert self.band_mismatch <= self.in_band, str(self)
+        assert self.band_mismatch <= max(2, MAX_BAND_FRACTION * self.mask_entries), \
+            f"too many in-band mask disagreements: {self}"
 
     def __str__(self):
-        return (f"rows={self.rows} max_abs={self.max_abs:.3e} rel_l2={self.rel_l2:.3e} "
-                f"band_mismatches={self.band_mismatch}")
+        return (f"heads={len(self.heads)} worst max_abs={self.max_abs:.3e} worst rel_l2={self.rel_l2:.3e} "
+                f"mask entries={self.mask_entries} in band={self.in_band} "
+                f"band mismatches={self.band_mismatch}")
+
+    def publish(self):
+        SESSION["mask_entries"] += self.mask_entries
+        SESSION["in_band"] += self.in_band
+        SESSION["band_mismatch"] += self.band_mismatch
+
+
+def _head_f64(qb, kb, vb, b, h):
+    q = bf16_bits_to_f64(qb[b, h])
+    k = bf16_bits_to_f64(kb[b, h])
+    v = bf16_bits_to_f64(vb[b, h]) if vb is not None else None
+    return q, k, v
+
+
+def check_full_masks(rep, qb, kb, b, h, beta, gpu_sel, gpu_counts):
+    """Every row's selection of slice (b, h) against the oracle's full proxy map
+    and thresholds (Eq. 3-5): equal outside the band |ŝ - τ| < 1e-4; the GPU's
+    counts are the popcounts of its masks."""
+    q, k, _ = _head_f64(qb, kb, None, b, h)
+    qbar, _, _ = pool_blocks(q)
+    kbar, _, _ = pool_blocks(k)
+    mu, sigma = row_stats_from_moments(qbar, *key_moments(kbar))
+    tau = thresholds(mu, sigma, beta)
+    s = proxy_logits(qbar, kbar)
+    sel_gpu = np.asarray(gpu_sel[b, h], dtype=bool)
+    N = s.shape[0]
+    ref = np.stack([select_global(s[i], tau[i]) for i in range(N)])
+    diff = sel_gpu != ref
+    near = np.abs(s - tau[:, None]) < BAND
+    outside = diff & ~near
+    assert not outside.any(), (f"mask mismatch outside the {BAND} band at head ({b},{h}): "
+                               f"{np.argwhere(outside)[:8].tolist()}")
+    rep.mask_entries += N * N
+    rep.in_band += int(near.sum())
+    rep.band_mismatch += int(diff.sum())
+    np.testing.assert_array_equal(gpu_counts[b, h], sel_gpu.sum(axis=1))
+
+
+def check_counts(qb, kb, b, h, beta, gpu_counts):
+    """sol_attn_stats of slice (b, h) against the oracle: each row's |S_i| lies
+    between the number of blocks above τ + band and above τ - band."""
+    q, k, _ = _head_f64(qb, kb, None, b, h)
+    qbar, _, _ = pool_blocks(q)
+    kbar, _, _ = pool_blocks(k)
+    mu, sigma = row_stats_from_moments(qbar, *key_moments(kbar))
+    tau = thresholds(mu, sigma, beta)
+    s = proxy_logits(qbar, kbar)
+    lo = (s >= tau[:, None] + BAND).sum(axis=1)
+    hi = (s >= tau[:, None] - BAND).sum(axis=1)
+    c = np.asarray(gpu_counts[b, h])
+    bad = np.nonzero((c < lo) | (c > hi))[0]
+    assert len(bad) == 0, f"head ({b},{h}) rows {bad[:8].tolist()}: counts {c[bad[:8]]} not in [{lo[bad[:8]]}, {hi[bad[:8]]}]"
+    SESSION["count_rows"] += len(c)
 
 
 def compare_head(rep, qb, kb, vb, b, h, beta, gpu_out, gpu_sel, gpu_counts, rows=None, exact_only=False,
                  dbg=None):
     """Compare one (b, h) slice on the given query blocks (default all)."""
-    q = bf16_bits_to_f64(qb[b, h])
-    k = bf16_bits_to_f64(kb[b, h])
-    v = bf16_bits_to_f64(vb[b, h])
+    q, k, v = _head_f64(qb, kb, vb, b, h)
     L = q.shape[0]
     N = -(-L // 64)
     rows = list(range(N)) if rows is None else list(rows)
@@ -71,8 +152,11 @@ def compare_head(rep, qb, kb, vb, b, h, beta, gpu_out, gpu_sel, gpu_counts, rows
     override_rows = []
     for i in rows:
         diff = np.nonzero(sel_gpu[i] != ref["sel"][i])[0]
+        s = proxy_row(ref["qbar"][i], ref["kbar"])
+        near = np.abs(s - ref["tau"][i]) < BAND
+        rep.mask_entries += N
+        rep.in_band += int(near.sum())
         if len(diff):
-            s = proxy_row(ref["qbar"][i], ref["kbar"])
             gap = np.abs(s[diff] - ref["tau"][i])
             assert (gap < BAND).all(), (f"mask mismatch outside the {BAND} band at head ({b},{h}) row {i}: "
                                         f"blocks {diff[gap >= BAND].tolist()} gap {gap[gap >= BAND].tolist()}")
@@ -97,12 +181,7 @@ def compare_head(rep, qb, kb, vb, b, h, beta, gpu_out, gpu_sel, gpu_counts, rows
             np.testing.assert_allclose(dbg["sigma"][b, h], ref["sigma"], rtol=2e-6, atol=BAND / 2)
     for i in rows:
         lo, hi = 64 * i, min(64 * i + 64, L)
-        g = gpu_out[b, h, lo:hi].astype(np.float64)
-        r = O[lo:hi]
-        rep.max_abs = max(rep.max_abs, float(np.abs(g - r).max()))
-        rep.num += float(((g - r) ** 2).sum())
-        rep.den += float((r ** 2).sum())
-        rep.rows += 1
+        rep.add_rows(b, h, gpu_out[b, h, lo:hi].astype(np.float64), O[lo:hi])
     return rep
 
 

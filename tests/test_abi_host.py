@@ -48,6 +48,10 @@ def test_argument_errors_without_gpu(lib):
     assert f(fake, fake, fake, fake, 1, 1, 128, 128, 32, 4, 1.0, 0, None, None) == -2       # block = 32
     assert f(fake, fake, fake, fake, 1, 1, 1 << 21, 128, 64, 4, 1.0, 0, None, None) == -2   # L too large
     assert f(fake, fake, fake, fake, 1, 1, 128, 128, 64, 0, 1.0, 0, None, None) == -1       # chunk = 0
+    # B*H beyond 65535 (gridDim.y of the pooling and moment kernels)
+    assert f(fake, fake, fake, ctypes.c_void_p(1 << 44), 1, 65536, 64, 64, 64, 4, 1.0, 0, None, None) == -2
+    assert f(fake, fake, fake, ctypes.c_void_p(1 << 44), 256, 257, 64, 64, 64, 4, 1.0, 0, None, None) == -2
+    assert "65535" in lib.sol_attn_error_string(-2).decode()
     assert f(fake, fake, fake, fake, 1, 1, 128, 128, 64, 4, math.nan, 0, None, None) == -1  # NaN beta
     assert f(mis, fake, fake, ctypes.c_void_p(0x90000), 1, 1, 128, 128, 64, 4, 1.0, 0, None, None) == -3
     assert f(fake, fake, fake, fake, 1, 1, 128, 128, 64, 4, 1.0, 0, None, None) == -1       # out aliases q

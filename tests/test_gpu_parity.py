@@ -9,8 +9,9 @@ import numpy as np
 import pytest
 
 import block_sparse_attention_moments_b200 as sa
-from parity_util import Report, compare_head, debug_numpy, run_gpu
-from synth import WORKLOADS, custom_fourier, fourier_inputs, gauss_inputs, offset_inputs, ramp_inputs
+from parity_util import Report, check_counts, check_full_masks, compare_head, debug_numpy, run_gpu
+from synth import (WORKLOADS, custom_fourier, fourier_inputs, gauss_inputs, near_block_constant_keys,
+                   offset_inputs, ramp_inputs)
 
 pytestmark = pytest.mark.gpu
 
@@ -23,7 +24,10 @@ def _lib():
     sa.lib()
 
 
-def _full_check(qb, kb, vb, beta, chunk, flags=0, heads=None, rows=None):
+def _full_check(qb, kb, vb, beta, chunk, flags=0, heads=None, rows=None, mask_heads=(), count_heads=()):
+    """Outputs of `heads` (all by default) on `rows` (all by default) against
+    the oracle, per head; every row's mask of `mask_heads`; the counts of
+    `count_heads` against the oracle's thresholds."""
     out, dbg, counts = run_gpu(qb, kb, vb, beta, chunk, flags=flags)
     sel = dbg.selection().cpu().numpy()
     dn = debug_numpy(dbg)
@@ -33,7 +37,13 @@ def _full_check(qb, kb, vb, beta, chunk, flags=0, heads=None, rows=None):
         b, h = divmod(bh, H)
         compare_head(rep, qb, kb, vb, b, h, beta, out, sel, counts, rows=rows,
                      exact_only=bool(flags & sa.FLAG_EXACT_ONLY), dbg=dn)
+    if not math.isinf(beta):
+        for bh in mask_heads:
+            check_full_masks(rep, qb, kb, *divmod(bh, H), beta, sel, counts)
+        for bh in count_heads:
+            check_counts(qb, kb, *divmod(bh, H), beta, counts)
     print(rep)
+    rep.publish()
     rep.check()
     return out, sel, rep
 
@@ -111,20 +121,54 @@ def test_image_shape():
     _full_check(qb, kb, vb, 1.0, wl.chunk, heads=full)
     rng = np.random.default_rng(5)
     rows = sorted(set(rng.integers(0, wl.N, size=6).tolist()) | {0, wl.N - 1})
-    _full_check(qb, kb, vb, 1.0, wl.chunk, heads=[bh for bh in range(B * H) if bh not in full][::5], rows=rows)
+    others = [bh for bh in range(B * H) if bh not in full]
+    # every other head: sampled outputs of every fifth, every row's mask of
+    # every fifth, the counts of all
+    _full_check(qb, kb, vb, 1.0, wl.chunk, heads=others[::5], rows=rows, mask_heads=others[2::5],
+                count_heads=range(B * H))
+
+
+_VIDEO = {}
+
+
+def _video_inputs(name):
+    if name not in _VIDEO:
+        _VIDEO.clear()
+        _VIDEO[name] = fourier_inputs(WORKLOADS[name])
+    return _VIDEO[name]
 
 
 @pytest.mark.parametrize("name,beta", [("wan", 1.0), ("wan", 0.75), ("wan", 1.5), ("hunyuan", 1.0),
-                                       ("hunyuan", -math.inf)])
+                                       ("hunyuan", 0.75), ("hunyuan", 1.5), ("hunyuan", -math.inf)])
 def test_video_shapes_sampled(name, beta):
-    # full-size launch (the bench's configuration); oracle on sampled query
-    # blocks of sampled heads, always including the ragged last block
+    # full-size launch (the bench's configuration); oracle outputs on sampled
+    # query blocks of sampled heads, always including the ragged last block;
+    # every row's mask of those heads; at beta = 1 the counts of every head
     wl = WORKLOADS[name]
-    qb, kb, vb = fourier_inputs(wl)
+    qb, kb, vb = _video_inputs(name)
     rng = np.random.default_rng(11)
     heads = sorted(set(rng.integers(0, wl.B * wl.H, size=3).tolist()) | {wl.B * wl.H - 1})
     rows = sorted(set(rng.integers(0, wl.N, size=4).tolist()) | {0, wl.N - 2, wl.N - 1})
-    _full_check(qb, kb, vb, beta, wl.chunk, heads=heads, rows=rows)
+    _full_check(qb, kb, vb, beta, wl.chunk, heads=heads, rows=rows, mask_heads=heads,
+                count_heads=range(wl.B * wl.H) if beta == 1.0 else ())
+
+
+@pytest.mark.parametrize("shape", ["tiny", "small"])
+@pytest.mark.parametrize("beta", [0.75, 1.0, 1.5])
+def test_mixed_selection_with_heavy_approximation(shape, beta):
+    # Keys nearly constant within each block (the block's first key plus 0.05
+    # N(0,1)): rows select some blocks and the zeroth-order term of the others
+    # carries a large share of the output (about half or more on these inputs,
+    # against ~1e-6 on the Fourier-feature workloads), so a slip in the
+    # approximation path fails here (method: proxy-score reuse, Eq. 8-10).
+    wl = WORKLOADS[shape]
+    qb, kb, vb = fourier_inputs(wl)
+    kb = near_block_constant_keys(kb, 0.05, seed=71)
+    out, sel, _ = _full_check(qb, kb, vb, beta, wl.chunk, mask_heads=range(wl.B * wl.H))
+    n_sel = sel.sum(axis=-1)
+    assert ((n_sel > 0) & (n_sel < wl.N)).any()        # mixed rows exist
+    exact, _, _ = run_gpu(qb, kb, vb, beta, wl.chunk, flags=sa.FLAG_EXACT_ONLY, debug=False)
+    assert np.linalg.norm(out - exact) > 0.1 * np.linalg.norm(out)
 
 
 @pytest.mark.parametrize("L,d,chunk", [(1, 128, 4), (64, 128, 1), (65, 64, 2), (127, 128, 4), (129, 64, 3),
