@@ -262,9 +262,10 @@ def run_role_profile(args):
 
 def run_ablation(args):
     """Approximation ablation (not a bench line): for each beta, the output of the
-    full method and of the exact-only variant (no approximation of unselected
-    blocks, same selection) against the select-all output of the same kernel,
-    as relative l2 error and mean per-row cosine similarity.  "Sol-Attn: ...",
+    full method, of its first-order extension and of the exact-only variant (no
+    approximation of unselected blocks, same selection) against the select-all
+    output of the same kernel, as relative l2 error and mean per-row cosine
+    similarity.  "Sol-Attn: ...",
     experiments: ablation of the proxy-score approximation."""
     import numpy as np
     import torch
@@ -273,6 +274,9 @@ def run_ablation(args):
     from synth import WORKLOADS
     wl = WORKLOADS[args.workload]
     qb, kb, vb = rank_inputs(wl, 0)
+    if args.ablation_keys == "near-block-constant":
+        from synth import near_block_constant_keys
+        kb = near_block_constant_keys(kb, 0.1, seed=73)
     dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
     q, k, v = dev(qb), dev(kb), dev(vb)
     dense = sa.forward(q, k, v, -math.inf, wl.chunk, flags=sa.FLAG_SELECT_ALL).float()
@@ -289,10 +293,14 @@ def run_ablation(args):
         counts = sa.stats(wl.B, wl.H, wl.L)
         density = counts.double().mean().item() / counts.shape[-1]
         o_exact = sa.forward(q, k, v, beta, wl.chunk, flags=sa.FLAG_EXACT_ONLY)
+        o_first = sa.forward(q, k, v, beta, wl.chunk, flags=sa.FLAG_FIRST_ORDER)
         rf, cf = compare(o_full)
         re, ce = compare(o_exact)
-        print(json.dumps({"mode": "ablation", "workload": wl.name, "beta": beta, "density": density,
+        r1, c1 = compare(o_first)
+        print(json.dumps({"mode": "ablation", "workload": wl.name, "keys": args.ablation_keys, "beta": beta,
+                          "density": density,
                           "approx": {"rel_l2_vs_dense": rf, "cosine_vs_dense": cf},
+                          "first_order": {"rel_l2_vs_dense": r1, "cosine_vs_dense": c1},
                           "exact_only": {"rel_l2_vs_dense": re, "cosine_vs_dense": ce}}), flush=True)
 
 
@@ -419,6 +427,8 @@ def main():
                     help="approximation ablation: full method and exact-only against select-all (not a bench line)")
     ap.add_argument("--ablation-betas", type=float, nargs="+", default=[0.75, 1.0, 1.5],
                     help="betas of --ablation and --density")
+    ap.add_argument("--ablation-keys", default="fourier", choices=["fourier", "near-block-constant"],
+                    help="keys of --ablation: the workload's, or each block's first key + 0.1 N(0,1)")
     ap.add_argument("--chunk-sweep", action="store_true",
                     help="outputs and times at several chunk sizes C (not a bench line)")
     ap.add_argument("--chunks", type=int, nargs="+", default=[1, 16, 64, 256, 1024])

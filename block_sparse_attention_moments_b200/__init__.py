@@ -17,7 +17,7 @@ import os
 from typing import Optional
 
 __all__ = [
-    "FLAG_SELECT_ALL", "FLAG_EXACT_ONLY", "FLAG_SYNC_CHECK", "FLAG_TEST_STALL", "SolAttnError", "lib", "lib_path",
+    "FLAG_SELECT_ALL", "FLAG_EXACT_ONLY", "FLAG_SYNC_CHECK", "FLAG_TEST_STALL", "FLAG_FIRST_ORDER", "SolAttnError", "lib", "lib_path",
     "forward", "stats", "forward_host", "stage_pool", "stage_threshold", "stage_fused",
     "workspace_bytes", "release", "kernels_per_forward", "DebugBuffers", "EXPORTED_SYMBOLS",
     "executed_flops", "BLOCK",
@@ -27,6 +27,7 @@ FLAG_SELECT_ALL = 0x1
 FLAG_EXACT_ONLY = 0x2
 FLAG_SYNC_CHECK = 0x4
 FLAG_TEST_STALL = 0x8   # failure-path test only: every bounded device wait runs out (see sol_attn.h)
+FLAG_FIRST_ORDER = 0x10  # first-order expansion for unselected blocks (extension; see sol_attn.h)
 BLOCK = 64
 
 _PKG = os.path.dirname(os.path.abspath(__file__))

@@ -101,6 +101,7 @@ __device__ unsigned long long g_profile[kProfileSlots];
 constexpr unsigned kFlagSelectAll = 1u;
 constexpr unsigned kFlagExactOnly = 2u;
 constexpr unsigned kFlagTestStall = 8u;    // routing publishes nothing: every role's wait runs out
+constexpr unsigned kFlagFirstOrder = 16u;  // unselected blocks: first-order expansion on exact tiles
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusDevice = 2u;     // a tile descriptor failed its range check
 
@@ -133,7 +134,7 @@ struct __align__(16) TileDesc {
   int ncols;            // 32, 64 or 128 (MMA N of S, K of PV)
   int flags;            // kDesc* bits
   int tail;             // column of the ragged block's approximation (weight n_tail), or -1
-  int pad;
+  int selbits;          // first-order mode: bit 2 h + b set when half h selected block b of the tile
 };
 constexpr int kDescFirst = 1;    // first tile of its item (PV overwrites O)
 constexpr int kDescLast = 2;     // last tile of its item
@@ -219,6 +220,7 @@ struct TileIter {
   int N, C, W;
   int nw;           // mask words per half
   bool has1, exact_only, first;
+  bool all_blocks;  // walk every block as exact (first-order mode), whatever the selection
   int lo, hi;       // current chunk [lo, hi)
   int jstart;       // the chunk's exact blocks run over [jstart, hi) then [lo, jstart)
   int seg;          // 0, 1: position in those two ranges; 2: exact blocks done
@@ -231,7 +233,7 @@ struct TileIter {
     int x = from;
     while (x < lim) {
       const int w = x >> 5;
-      const uint32_t u = (m0[w] | m1[w]) & (0xFFFFFFFFu << (x & 31));
+      const uint32_t u = (all_blocks ? 0xFFFFFFFFu : (m0[w] | m1[w])) & (0xFFFFFFFFu << (x & 31));
       if (u) {
         const int jj = (w << 5) + __ffs(u) - 1;
         return jj < lim ? jj : lim;
@@ -271,6 +273,7 @@ struct TileIter {
     nw = (N_ + 31) >> 5;
     has1 = has1_;
     exact_only = exact_only_;
+    all_blocks = false;
     first = true;
     chunks_left = (N_ + C_ - 1) / C_;
     lo = (i0 / C_) * C_;
@@ -362,7 +365,9 @@ __device__ __forceinline__ float exp2_neg_int(float k) {
   return (ki >= 126) ? 0.f : __int_as_float((127 - ki) << 23);
 }
 
-template <int D>
+// FO: the first-order mode (kFlagFirstOrder) is a separate instantiation, so
+// that its extra per-tile work does not enter the default kernel's code.
+template <int D, bool FO>
 __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
     sol_attn_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kb,
@@ -383,6 +388,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
   constexpr uint32_t CB = 16384;           // bytes per 64-column block of a 128-row tile
   volatile int* abort_flag = &ctl.abort;
   const bool exact_only = (p.flags & kFlagExactOnly) != 0;
+  constexpr bool first_order = FO;
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -559,7 +565,8 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
         publish();
       } else {
         TileIter it;
-        it.init(sl, p.N, p.chunk, p.W, 2 * pair, 2 * pair + 1 < p.N, exact_only);
+        it.init(sl, p.N, p.chunk, p.W, 2 * pair, 2 * pair + 1 < p.N, exact_only || first_order);
+        it.all_blocks = first_order;
         Tile t, tn;
         bool have = it.next(t);
         bool first_desc = true;
@@ -580,7 +587,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
                 const int jx = (g < 2) ? t.ja : t.jb;
                 const int nv = min(max(p.L - (64 * jx + 32 * (g & 1)), 0), 32);
                 const uint32_t range = (nv >= 32) ? 0xFFFFFFFFu : ((1u << nv) - 1u);
-                bits = mask_bit(sl.mask[h], jx) ? range : 0u;
+                bits = (first_order || mask_bit(sl.mask[h], jx)) ? range : 0u;
               }
             }
             dsc->bits[h][g] = bits;
@@ -593,6 +600,15 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
             dsc->ncols = t.ncols;
             dsc->flags = (t.first ? kDescFirst : 0) | (have_next ? 0 : kDescLast) | (t.kind == 0 ? kDescApprox : 0);
             dsc->tail = (tail_col >= 0 && tail_col < t.ncols) ? tail_col : -1;
+            int sb = 0xF;
+            if (first_order && t.kind == 1) {
+              sb = 0;
+              for (int h = 0; h < 2; ++h) {
+                if (mask_bit(sl.mask[h], t.ja)) sb |= 1 << (2 * h);
+                if (t.jb >= 0 && mask_bit(sl.mask[h], t.jb)) sb |= 2 << (2 * h);
+              }
+            }
+            dsc->selbits = sb;
           }
           publish();
           t = tn;
@@ -791,6 +807,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
       const TileDesc& dsc = ctl.ring[r % kRing];
       const uint4 bw = *reinterpret_cast<const uint4*>(dsc.bits[half]);
       const int ncols = dsc.ncols, dflags = dsc.flags, tail_col = dsc.tail, dbh = dsc.bh, dpair = dsc.pair;
+      const int selbits = dsc.selbits;
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.ring_empty[r % kRing]);
       if (dflags & kDescEnd) break;
@@ -845,6 +862,31 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
           const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
           float m_cur = m_own;
           float2 ra = make_float2(0.f, 0.f), rb = make_float2(0.f, 0.f);
+          // First-order mode: a block this row's half did not select is
+          // expanded around its row-wise mean score c (the mean of the exact
+          // scores over the block's valid keys, equal to q.K̄_j/sqrt(d)):
+          // weight 2^(c - m) (1 + (s - c)) in natural-log units of s and c.
+          const bool lin0 = first_order && !((selbits >> (2 * half)) & 1);
+          const bool lin1 = first_order && ncols == 128 && !((selbits >> (2 * half + 1)) & 1);
+          float xc0 = 0.f, xc1 = 0.f;   // raw-score means of the tile's two blocks
+          if (__any_sync(0xFFFFFFFFu, lin0 || lin1)) {
+#pragma unroll 1
+            for (int g = 0; g < ng; ++g) {
+              float xv[32];
+              tmem_ld_x32f(tS + 32 * g, xv);
+              tmem_ld_wait();
+              reg_fence32(xv);
+              const uint32_t bits = gb(g);
+              float sum = 0.f;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) sum += ((bits >> e) & 1u) ? xv[e] : 0.f;
+              if (g < 2) xc0 += sum; else xc1 += sum;
+            }
+            const int n0 = __popc(gb(0)) + (ng > 1 ? __popc(gb(1)) : 0);
+            const int n1 = (ng > 2) ? __popc(gb(2)) + __popc(gb(3)) : 0;
+            xc0 = n0 ? xc0 / static_cast<float>(n0) : 0.f;
+            xc1 = n1 ? xc1 / static_cast<float>(n1) : 0.f;
+          }
 #pragma unroll 1
           for (int g = 0; g < ng; ++g) {
             float xv[32];
@@ -867,6 +909,19 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
             const float2 of2 = make_float2(boost - mref, boost - mref);
             SA_PROF(const unsigned long long te0 = clock64();)
             uint32_t pk[16];
+            const bool lin = (g < 2) ? lin0 : lin1;
+            if (lin) {   // first-order weights of an unselected block (warp-uniform: a warp's rows share a half)
+              const float xc = (g < 2) ? xc0 : xc1;
+              const float ec = ex2_approx(fmaf(xc, p.scale_log2, boost - mref));
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float w0 = (xv[e] == -INFINITY) ? 0.f : ec * fmaf(xv[e] - xc, p.inv_sqrt_d, 1.f);
+                const float w1 = (xv[e + 1] == -INFINITY) ? 0.f : ec * fmaf(xv[e + 1] - xc, p.inv_sqrt_d, 1.f);
+                ra.x += w0;
+                ra.y += w1;
+                pk[e >> 1] = pack_bf16x2(w0, w1);
+              }
+            } else {
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               const float2 y0 = __ffma2_rn(make_float2(xv[e], xv[e + 1]), sc2, of2);
@@ -883,6 +938,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
               pk[(e >> 1) + 1] = pack_bf16x2(q1.x, q1.y);
               pk[(e >> 1) + 2] = pack_bf16x2(q2.x, q2.y);
               pk[(e >> 1) + 3] = pack_bf16x2(q3.x, q3.y);
+            }
             }
             tmem_st_x16(tS + 16 * g, pk);
             SA_PROF(prof[kPrSmExp] += clock64() - te0;)

@@ -342,13 +342,18 @@ int launch_fused(Workspace& w, const void* q, const void* k, const void* v, void
   static bool attr_set[kMaxDevices] = {false};   // the attribute is set per device
   if (dev < 0 || dev >= kMaxDevices) return fail(SOL_ATTN_ERR_UNSUPPORTED, "device index %d too large", dev);
   if (!attr_set[dev]) {
-    CUDA_TRY(cudaFuncSetAttribute(sol_attn_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    CUDA_TRY(cudaFuncSetAttribute(sol_attn_fused_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kFusedSmemBytes)));
+    CUDA_TRY(cudaFuncSetAttribute(sol_attn_fused_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(kFusedSmemBytes)));
     attr_set[dev] = true;
   }
   CUDA_TRY(cudaMemsetAsync(w.counter, 0, sizeof(unsigned), st));
   const int grid = std::min(p.num_items, nsm);
-  sol_attn_fused_kernel<D><<<grid, kThreads, kFusedSmemBytes, st>>>(tq, tk, tv, tkb, tkl, tvb, p);
+  if (flags & SOL_ATTN_FLAG_FIRST_ORDER)
+    sol_attn_fused_kernel<D, true><<<grid, kThreads, kFusedSmemBytes, st>>>(tq, tk, tv, tkb, tkl, tvb, p);
+  else
+    sol_attn_fused_kernel<D, false><<<grid, kThreads, kFusedSmemBytes, st>>>(tq, tk, tv, tkb, tkl, tvb, p);
   CUDA_TRY(cudaGetLastError());
   return SOL_ATTN_OK;
 }
@@ -419,6 +424,15 @@ int noalloc_base(int dev, char** out) {
   return SOL_ATTN_OK;
 }
 
+int check_flags(unsigned flags) {
+  if ((flags & SOL_ATTN_FLAG_FIRST_ORDER) && (flags & SOL_ATTN_FLAG_EXACT_ONLY))
+    return fail(SOL_ATTN_ERR_ARG, "FIRST_ORDER and EXACT_ONLY exclude each other");
+  if (flags & ~(SOL_ATTN_FLAG_SELECT_ALL | SOL_ATTN_FLAG_EXACT_ONLY | SOL_ATTN_FLAG_SYNC_CHECK |
+                SOL_ATTN_FLAG_TEST_STALL | SOL_ATTN_FLAG_FIRST_ORDER))
+    return fail(SOL_ATTN_ERR_ARG, "unknown flag bits 0x%x", flags);
+  return SOL_ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -427,6 +441,7 @@ int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, 
                         int chunk, float beta, unsigned flags, const sol_attn_debug* dbg, void* stream) {
   int rc;
   if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if ((rc = check_flags(flags))) return rc;
   if (chunk < 1) return fail(SOL_ATTN_ERR_ARG, "chunk must be >= 1 (got %d)", chunk);
   if (std::isnan(beta)) return fail(SOL_ATTN_ERR_ARG, "beta is NaN");
   if (!out) return fail(SOL_ATTN_ERR_ARG, "out is NULL");
@@ -476,6 +491,7 @@ int sol_attn_stage_fused(const void* q, const void* k, const void* v, void* out,
                          int chunk, unsigned flags, const sol_attn_debug* dbg, void* stream) {
   int rc;
   if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if ((rc = check_flags(flags))) return rc;
   if (chunk < 1) return fail(SOL_ATTN_ERR_ARG, "chunk must be >= 1 (got %d)", chunk);
   if (!out) return fail(SOL_ATTN_ERR_ARG, "out is NULL");
   if ((rc = check_io(q, k, v, out, B, H, L, d))) return rc;

@@ -48,7 +48,8 @@ extern "C" {
 
 typedef enum sol_attn_status {
   SOL_ATTN_OK = 0,
-  SOL_ATTN_ERR_ARG = -1,          /* null pointer, non-positive size, NaN beta, chunk < 1 */
+  SOL_ATTN_ERR_ARG = -1,          /* null pointer, non-positive size, NaN beta, chunk < 1,
+                                     unknown or conflicting flags */
   SOL_ATTN_ERR_UNSUPPORTED = -2,  /* d not in {64,128}, block != 64, L too large, B*H > 65535,
                                      not sm_100 */
   SOL_ATTN_ERR_ALIGN = -3,        /* a tensor base address is not 16-byte aligned */
@@ -72,6 +73,13 @@ typedef enum sol_attn_status {
                                           gives up after 1 ms, the kernel exits cleanly and
                                           the status word reports SOL_ATTN_ERR_TIMEOUT; out
                                           is left unwritten */
+#define SOL_ATTN_FLAG_FIRST_ORDER 0x10u /* extension (the method keeps the zeroth order only):
+                                          every block goes through the exact tile path and a
+                                          block the row did not select gets the first-order
+                                          expansion of Eq. 8 around its row-wise mean score
+                                          c = q.K̄_j/sqrt(d), weight e^c (1 + (s - c)) per key,
+                                          instead of the zeroth-order e^c; costs as much as
+                                          the select-all mode.  Excludes EXACT_ONLY. */
 
 /* Optional device buffers filled by sol_attn_forward_ex (any member may be NULL).
  * Shapes use N = ceil(L/64); all are row-major and owned by the caller. */

@@ -46,10 +46,21 @@ def run_gpu(qb, kb, vb, beta, chunk, flags=0, debug=True):
     return out.float().cpu().numpy(), dbg, counts.cpu().numpy()
 
 
+# The first-order extension (not one of the workload's configurations) weights
+# a skipped block's keys by e^c (1 + (s - c)): unlike softmax weights these
+# are not confined to [0, 1] of the row maximum and take both signs, so the
+# bf16 rounding of P (relative 2^-9 per weight) gives an absolute output error
+# that scales with sum |w| |v| / sum w instead of |v|.  Its max-abs bound is
+# raised by half (measured worst: 2.2e-2 with every block expanded on the
+# tiny shape); the rel-l2 bound is unchanged.
+MAX_ABS_FIRST_ORDER = 3e-2
+
+
 class Report:
     """Output errors per (batch, head) slice and mask agreement of one test."""
 
-    def __init__(self):
+    def __init__(self, max_abs=MAX_ABS):
+        self.max_abs_bound = max_abs
         self.heads = {}           # (b, h) -> [max_abs, sum sq err, sum sq ref, rows]
         self.mask_entries = 0
         self.in_band = 0
@@ -75,7 +86,7 @@ class Report:
         return max((v[1] for v in self.per_head().values()), default=0.0)
 
     def check(self):
-        bad = {k: v for k, v in self.per_head().items() if v[0] > MAX_ABS or v[1] > REL_L2}
+        bad = {k: v for k, v in self.per_head().items() if v[0] > self.max_abs_bound or v[1] > REL_L2}
         assert not bad, f"heads over tolerance (max-abs, rel-l2, rows): {bad}; {self}"
         assert self.band_mismatch <= self.in_band, str(self)
         assert self.band_mismatch <= max(2, MAX_BAND_FRACTION * self.mask_entries), \
@@ -141,13 +152,13 @@ def check_counts(qb, kb, b, h, beta, gpu_counts):
 
 
 def compare_head(rep, qb, kb, vb, b, h, beta, gpu_out, gpu_sel, gpu_counts, rows=None, exact_only=False,
-                 dbg=None):
+                 dbg=None, taylor_order=0):
     """Compare one (b, h) slice on the given query blocks (default all)."""
     q, k, v = _head_f64(qb, kb, vb, b, h)
     L = q.shape[0]
     N = -(-L // 64)
     rows = list(range(N)) if rows is None else list(rows)
-    ref = sol_attn_head(q, k, v, beta, exact_only=exact_only, rows=rows)
+    ref = sol_attn_head(q, k, v, beta, exact_only=exact_only, rows=rows, taylor_order=taylor_order)
     sel_gpu = np.asarray(gpu_sel[b, h], dtype=bool)
     override_rows = []
     for i in rows:
@@ -165,7 +176,8 @@ def compare_head(rep, qb, kb, vb, b, h, beta, gpu_out, gpu_sel, gpu_counts, rows
         assert gpu_counts[b, h, i] == sel_gpu[i].sum()
     O = ref["O"]
     if override_rows:   # evaluate those rows with the GPU's (equally valid) selection
-        alt = sol_attn_head(q, k, v, beta, exact_only=exact_only, rows=override_rows, sel_override=sel_gpu)
+        alt = sol_attn_head(q, k, v, beta, exact_only=exact_only, rows=override_rows, sel_override=sel_gpu,
+                            taylor_order=taylor_order)
         for i in override_rows:
             lo, hi = 64 * i, min(64 * i + 64, L)
             O[lo:hi] = alt["O"][lo:hi]

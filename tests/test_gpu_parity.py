@@ -9,7 +9,8 @@ import numpy as np
 import pytest
 
 import block_sparse_attention_moments_b200 as sa
-from parity_util import Report, check_counts, check_full_masks, compare_head, debug_numpy, run_gpu
+from parity_util import (MAX_ABS, MAX_ABS_FIRST_ORDER, Report, check_counts, check_full_masks, compare_head,
+                         debug_numpy, run_gpu)
 from synth import (WORKLOADS, custom_fourier, fourier_inputs, gauss_inputs, near_block_constant_keys,
                    offset_inputs, ramp_inputs)
 
@@ -31,12 +32,13 @@ def _full_check(qb, kb, vb, beta, chunk, flags=0, heads=None, rows=None, mask_he
     out, dbg, counts = run_gpu(qb, kb, vb, beta, chunk, flags=flags)
     sel = dbg.selection().cpu().numpy()
     dn = debug_numpy(dbg)
-    rep = Report()
+    rep = Report(MAX_ABS_FIRST_ORDER if flags & sa.FLAG_FIRST_ORDER else MAX_ABS)
     B, H = qb.shape[:2]
     for bh in (range(B * H) if heads is None else heads):
         b, h = divmod(bh, H)
         compare_head(rep, qb, kb, vb, b, h, beta, out, sel, counts, rows=rows,
-                     exact_only=bool(flags & sa.FLAG_EXACT_ONLY), dbg=dn)
+                     exact_only=bool(flags & sa.FLAG_EXACT_ONLY), dbg=dn,
+                     taylor_order=1 if flags & sa.FLAG_FIRST_ORDER else 0)
     if not math.isinf(beta):
         for bh in mask_heads:
             check_full_masks(rep, qb, kb, *divmod(bh, H), beta, sel, counts)
@@ -291,3 +293,44 @@ def test_bounded_wait_runs_out_and_the_next_forward_is_clean():
     assert "timed out" in str(e.value)
     torch.cuda.synchronize()
     _full_check(qb, kb, vb, 1.0, wl.chunk)
+
+
+@pytest.mark.parametrize("beta", [0.75, 1.0, 1.5, math.inf])
+@pytest.mark.parametrize("case", ["tiny", "small", "small_blocky", "ragged"])
+def test_first_order_flag(case, beta):
+    # Extension of the proxy-score reuse (Eq. 8): unselected blocks take the
+    # first-order expansion around their row-wise mean score; against the
+    # oracle's taylor_order=1 on identical inputs.
+    if case == "ragged":
+        qb, kb, vb = custom_fourier(1, 2, (1, 1, 1000), 128, 2.0, seed=401)
+        chunk = 5
+    else:
+        wl = WORKLOADS["tiny" if case == "tiny" else "small"]
+        qb, kb, vb = fourier_inputs(wl)
+        chunk = wl.chunk
+        if case == "small_blocky":
+            kb = near_block_constant_keys(kb, 0.1, seed=73)
+    _full_check(qb, kb, vb, beta, chunk, flags=sa.FLAG_FIRST_ORDER)
+
+
+def test_first_order_is_closer_to_dense_on_near_constant_keys():
+    # With keys K̄_j + eps R the zeroth-order error is O(eps), the first-order O(eps^2)
+    wl = WORKLOADS["small"]
+    qb, kb, vb = fourier_inputs(wl)
+    kb = near_block_constant_keys(kb, 0.1, seed=73)
+    dense, _, _ = run_gpu(qb, kb, vb, -math.inf, wl.chunk, debug=False)
+    zero, _, _ = run_gpu(qb, kb, vb, 1.0, wl.chunk, debug=False)
+    first, _, _ = run_gpu(qb, kb, vb, 1.0, wl.chunk, flags=sa.FLAG_FIRST_ORDER, debug=False)
+    e0 = np.linalg.norm(zero - dense) / np.linalg.norm(dense)
+    e1 = np.linalg.norm(first - dense) / np.linalg.norm(dense)
+    print(f"rel-l2 vs select-all: zeroth order {e0:.2e}, first order {e1:.2e}")
+    assert e1 < 0.5 * e0
+
+
+def test_conflicting_flags_are_rejected():
+    from parity_util import to_device
+    wl = WORKLOADS["tiny"]
+    q, k, v = (to_device(x) for x in fourier_inputs(wl))
+    with pytest.raises(sa.SolAttnError) as e:
+        sa.forward(q, k, v, 1.0, wl.chunk, flags=sa.FLAG_FIRST_ORDER | sa.FLAG_EXACT_ONLY)
+    assert e.value.code == -1
