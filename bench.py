@@ -257,6 +257,10 @@ def run_role_profile(args):
                           "issuer_cycles_per_tile": {k2: round(prof[k2] / tiles, 1) for k2 in
                                                      ("s.issue", "s.wait_buffer", "s.wait_k", "s.wait_desc",
                                                       "pv.issue", "pv.wait_p", "pv.wait_v", "pv.wait_desc")},
+                          "other_roles_cycles_per_tile": {k2: round(prof[k2] / tiles, 1) for k2 in
+                                                          ("sched.walk", "sched.descriptor", "sched.wait_ring",
+                                                           "route.item", "route.wait_item_empty", "k.wait_stage",
+                                                           "v.wait_stage")},
                           "rescales": prof["softmax.rescales"]}), flush=True)
 
 

@@ -235,7 +235,7 @@ PROFILE_SLOTS = (
     "softmax.pass", "softmax.meet", "softmax.epilogue", "softmax.tiles", "softmax.rescales",
     "sched.wait_item", "sched.wait_ring",
     "total.route", "total.k", "total.v", "total.s", "total.pv", "total.softmax", "total.sched",
-    "softmax.tmem_load", "softmax.exp_block",
+    "softmax.tmem_load", "softmax.exp_block", "sched.walk", "sched.descriptor", "route.item",
 )
 
 

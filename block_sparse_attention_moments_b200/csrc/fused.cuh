@@ -88,7 +88,7 @@ enum ProfSlot : int {
   kPrPvDesc, kPrPvP, kPrPvV, kPrPvIssue,
   kPrSmDesc, kPrSmS, kPrSmHand, kPrSmO, kPrSmX, kPrSmPass, kPrSmMeet, kPrSmEpi, kPrSmTiles, kPrSmRescales,
   kPrSchedItem, kPrSchedRing,
-  kPrTotRoute, kPrTotK, kPrTotV, kPrTotS, kPrTotPv, kPrTotSm, kPrTotSched, kPrSmLd, kPrSmExp, kPrSlots
+  kPrTotRoute, kPrTotK, kPrTotV, kPrTotS, kPrTotPv, kPrTotSm, kPrTotSched, kPrSmLd, kPrSmExp, kPrSchedNext, kPrSchedDesc, kPrRouteItem, kPrSlots
 };
 constexpr int kProfileSlots = 48;
 static_assert(kPrSlots <= kProfileSlots, "profile slots");
@@ -467,6 +467,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
         }
         break;
       }
+      SA_PROF(const unsigned long long tr0 = clock64();)
       const int bh = item / p.num_pairs;
       const int pair = item - bh * p.num_pairs;
       const int i0 = 2 * pair, i1 = 2 * pair + 1;
@@ -487,15 +488,23 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
         const int j = 32 * g + lane;
         bool s0 = false, s1 = false;
         if (j < p.N) {
+          // the key's 128 floats (L2-resident) in batches of 8 x 16 bytes, all
+          // loads of a batch in flight before its products
           const float4* kr = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
-#pragma unroll 2
-          for (int c4 = 0; c4 < D / 4; ++c4) {
-            const float4 x = __ldg(kr + c4);
-            const float4 qa = *reinterpret_cast<const float4*>(&ctl.qbar[0][4 * c4]);
-            const float4 qb4 = *reinterpret_cast<const float4*>(&ctl.qbar[1][4 * c4]);
-            a0 = fmaf(qa.x, x.x, a0); a1 = fmaf(qa.y, x.y, a1); a2 = fmaf(qa.z, x.z, a2); a3 = fmaf(qa.w, x.w, a3);
-            b0 = fmaf(qb4.x, x.x, b0); b1 = fmaf(qb4.y, x.y, b1); b2 = fmaf(qb4.z, x.z, b2); b3 = fmaf(qb4.w, x.w, b3);
+#pragma unroll 1
+          for (int c0 = 0; c0 < D / 4; c0 += 8) {
+            float4 xs[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) xs[u] = __ldg(kr + c0 + u);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float4 x = xs[u];
+              const float4 qa = *reinterpret_cast<const float4*>(&ctl.qbar[0][4 * (c0 + u)]);
+              const float4 qb4 = *reinterpret_cast<const float4*>(&ctl.qbar[1][4 * (c0 + u)]);
+              a0 = fmaf(qa.x, x.x, a0); a1 = fmaf(qa.y, x.y, a1); a2 = fmaf(qa.z, x.z, a2); a3 = fmaf(qa.w, x.w, a3);
+              b0 = fmaf(qb4.x, x.x, b0); b1 = fmaf(qb4.y, x.y, b1); b2 = fmaf(qb4.z, x.z, b2); b3 = fmaf(qb4.w, x.w, b3);
+            }
           }
           const float d0 = (a0 + a1) + (a2 + a3);
           const float d1 = (b0 + b1) + (b2 + b3);
@@ -526,6 +535,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
         }
       }
       __syncwarp();
+      SA_PROF(prof[kPrRouteItem] += clock64() - tr0;)
       if (lane == 0) mbar_arrive(&ctl.item_full[s]);   // release: masks and item visible
     }
   } else if (warp == kWarpSched) {
@@ -571,9 +581,12 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
         bool have = it.next(t);
         bool first_desc = true;
         while (have) {
+          SA_PROF(const unsigned long long tn0 = clock64();)
           const bool have_next = it.next(tn);
+          SA_PROF(prof[kPrSchedNext] += clock64() - tn0;)
           if (!first_desc && !(dsc = claim())) break;
           first_desc = false;
+          SA_PROF(const unsigned long long td0 = clock64();)
           // lanes 0-7 each compute one (half, 32-column group) validity word
           if (lane < 8) {
             const int g = lane >> 1, h = lane & 1;
@@ -611,6 +624,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
             dsc->selbits = sb;
           }
           publish();
+          SA_PROF(prof[kPrSchedDesc] += clock64() - td0;)
           t = tn;
           have = have_next;
         }
