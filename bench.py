@@ -414,6 +414,134 @@ def run_speedup_sweep(args):
         del q, k, v
 
 
+def run_routing_cost(args):
+    """Routing-cost report (not a bench line): the method's routing against a
+    materialised top-k router, on the workload's shape.  "Sol-Attn: ...",
+    experiments: routing latency against top-k / top-p routers that materialise
+    and traverse the proxy map (Fig. 5b/5c).
+
+    method  exposed: the moment kernels (key mean and covariance, then mu_i,
+            sigma_i and tau_i for every query block; CUDA events).  The routing
+            dot products and threshold tests run inside the fused kernel beside
+            its tiles; their routing-warp busy cycles (profiling build), summed
+            over the SMs and divided by SMs x SM clock, are reported apart.
+    top-k   the whole proxy map of every head written to HBM, then each row's
+            k largest blocks selected (k = the row-average |S_i| of the method
+            at this beta, so both keep the same number of blocks); CUDA events.
+    Workspace bytes of each are reported beside the times."""
+    os.environ["SOL_ATTN_PROFILE"] = "1"
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_moments_b200 as sa
+    from synth import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    qb, kb, vb = rank_inputs(wl, 0)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = dev(qb), dev(kb), dev(vb)
+    B, H, L, d, N = 1, wl.H, wl.L, wl.d, wl.N
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    out = torch.empty_like(q)
+
+    def timed(fn, reps=5):
+        for _ in range(2):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    sa.stage_pool(q, k, v)
+    thr_ms = timed(lambda: sa.stage_threshold(B, H, L, d, args.beta))
+    # one full forward in the profiling build for the in-kernel routing cycles
+    sa.forward(q, k, v, args.beta, wl.chunk)
+    sa.profile_read(reset=True)
+    sa.forward(q, k, v, args.beta, wl.chunk)
+    prof = sa.profile_read(reset=True)
+    counts = sa.stats(B, H, L)
+    kk = int(round(counts.double().mean().item()))
+    clk_hz = 1e6 * float(os.environ.get("SOL_ATTN_SM_MHZ", "1965"))
+    route_ms = prof["route.item"] / nsm / clk_hz * 1e3
+    sa.stage_pool(q, k, v)
+    topk_ms = timed(lambda: sa.topk_route(B, H, L, d, kk))
+    method_bytes = B * H * N * 4 + B * H * (d + d * d) * 8          # thresholds + key moments
+    topk_bytes = B * H * N * N * 4                                     # the materialised map
+    # The top-k router runs as its own kernels before attention can start; of
+    # the method's routing only the moment kernels do, the dot products and
+    # threshold tests run inside the fused kernel beside its tiles.
+    print(json.dumps({"mode": "routing_cost", "workload": wl.name, "beta": args.beta, "blocks_kept_per_row": kk,
+                      "method": {"exposed_ms": thr_ms, "workspace_bytes": method_bytes,
+                                 "in_kernel_routing_warp_ms_equivalent": route_ms},
+                      "topk_materialised": {"exposed_ms": topk_ms, "workspace_bytes": topk_bytes},
+                      "exposed_time_ratio_topk_over_method": topk_ms / thr_ms,
+                      "workspace_ratio_topk_over_method": topk_bytes / method_bytes,
+                      "sm_clock_mhz_assumed": clk_hz / 1e6}), flush=True)
+
+
+def run_all_configs(args):
+    """Per-configuration report (not a bench line): for each video shape and
+    beta of the workload list, and the select-all mode, the forward time (the
+    three stages, CUDA events, inputs larger than L2), executed TFLOPS by the
+    method's accounting, the fused kernel's fraction of the measured bf16 burst
+    peak and the speedup over the same shape's select-all mode."""
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_moments_b200 as sa
+    from synth import WORKLOADS
+    peaks, _ = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    for name in args.configs:
+        wl = WORKLOADS[name]
+        qb, kb, vb = rank_inputs(wl, 0)
+        dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+        q, k, v = dev(qb), dev(kb), dev(vb)
+        out = torch.empty_like(q)
+        B, H, L, d, N = 1, wl.H, wl.L, wl.d, wl.N
+
+        def one(beta, flags, reps):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            tot = [0.0, 0.0, 0.0]
+            for r in range(reps + 3):
+                ev[0].record()
+                sa.stage_pool(q, k, v)
+                ev[1].record()
+                sa.stage_threshold(B, H, L, d, beta, flags=flags)
+                ev[2].record()
+                sa.stage_fused(q, k, v, out, wl.chunk, flags=flags)
+                ev[3].record()
+                torch.cuda.synchronize()
+                if r >= 3:
+                    for i in range(3):
+                        tot[i] += ev[i].elapsed_time(ev[i + 1]) / reps
+            counts = sa.stats(B, H, L)
+            pairs = int(counts.to(torch.int64).sum().item())
+            return tot, pairs
+
+        dense_t, dense_pairs = one(-math.inf, sa.FLAG_SELECT_ALL, 2)
+        dense_ms = sum(dense_t)
+        rows = [("select-all", dense_t, dense_pairs, -math.inf)]
+        for beta in wl.betas:
+            if math.isinf(beta):
+                continue
+            t, pairs = one(beta, 0, args.steps)
+            rows.append((beta, t, pairs, beta))
+        for label, t, pairs, beta in rows:
+            ms = sum(t)
+            approx = not math.isinf(beta)
+            fl = sa.executed_flops(pairs, B, H, L, d, approx=approx)
+            print(json.dumps({"mode": "config", "workload": wl.name, "beta": label, "density": pairs / (B * H * N * N),
+                              "ms_per_forward": ms, "stage_ms": {"pool": t[0], "threshold": t[1], "fused": t[2]},
+                              "executed_tflops": fl / (ms * 1e-3) / 1e12,
+                              "fused_frac_of_burst_peak": fl / (t[2] * 1e-3) / 1e12 / peak,
+                              "speedup_vs_select_all": dense_ms / ms}), flush=True)
+        del q, k, v, out
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -444,11 +572,20 @@ def main():
     ap.add_argument("--sweep-betas", type=float, nargs="+", default=[0.84, 1.28, 1.64],
                     help="about 80%%, 90%% and 95%% sparsity on Gaussian proxy logits")
     ap.add_argument("--sweep-heads", type=int, default=8)
+    ap.add_argument("--all-configs", action="store_true",
+                    help="time, TFLOPS, fraction of peak and speedup for every video shape and beta (not a bench line)")
+    ap.add_argument("--configs", nargs="+", default=["wan", "hunyuan"])
+    ap.add_argument("--routing-cost", action="store_true",
+                    help="method's routing against a materialised top-k router (not a bench line)")
     ap.add_argument("--role-profile", action="store_true",
                     help="run the profiling build (libsol_attn_profile.so) and print per-role cycle accounting")
     args = ap.parse_args()
     if args.role_profile:
         return run_role_profile(args)
+    if args.routing_cost:
+        return run_routing_cost(args)
+    if args.all_configs:
+        return run_all_configs(args)
     if args.ablation:
         return run_ablation(args)
     if args.density:

@@ -19,7 +19,7 @@ from typing import Optional
 __all__ = [
     "FLAG_SELECT_ALL", "FLAG_EXACT_ONLY", "FLAG_SYNC_CHECK", "FLAG_TEST_STALL", "FLAG_FIRST_ORDER", "SolAttnError", "lib", "lib_path",
     "forward", "stats", "forward_host", "stage_pool", "stage_threshold", "stage_fused",
-    "workspace_bytes", "release", "kernels_per_forward", "DebugBuffers", "EXPORTED_SYMBOLS",
+    "workspace_bytes", "release", "kernels_per_forward", "DebugBuffers", "EXPORTED_SYMBOLS", "topk_route",
     "executed_flops", "BLOCK",
 ]
 
@@ -42,7 +42,7 @@ EXPORTED_SYMBOLS = (
     "sol_attn_stage_pool", "sol_attn_stage_threshold", "sol_attn_stage_fused",
     "sol_attn_workspace_bytes", "sol_attn_release", "sol_attn_error_string",
     "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc", "sol_attn_profile_read",
-    "sol_attn_noalloc_status",
+    "sol_attn_noalloc_status", "sol_attn_topk_route",
 )
 
 
@@ -88,10 +88,11 @@ def lib():
     L.sol_attn_forward_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.sol_attn_profile_read.argtypes = [vp, i, i]
     L.sol_attn_noalloc_status.argtypes = [vp]
+    L.sol_attn_topk_route.argtypes = [i, i, i, i, i, i, vp, vp]
     for name in ("sol_attn_forward", "sol_attn_forward_ex", "sol_attn_stats", "sol_attn_forward_host",
                  "sol_attn_stage_pool", "sol_attn_stage_threshold", "sol_attn_stage_fused", "sol_attn_release",
                  "sol_attn_kernels_per_forward", "sol_attn_forward_noalloc", "sol_attn_profile_read",
-                 "sol_attn_noalloc_status"):
+                 "sol_attn_noalloc_status", "sol_attn_topk_route"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -219,6 +220,19 @@ def stage_fused(q, k, v, out, chunk: int, *, flags: int = 0, debug: Optional[Deb
     _check(lib().sol_attn_stage_fused(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, L, d, BLOCK,
                                       int(chunk), int(flags), dbg, _stream_handle(stream)))
     return out
+
+
+def topk_route(B: int, H: int, L: int, d: int, k: int, stream=None):
+    """Comparison top-k router (measurement aid): from the pooled Q̄, K̄ of the
+    last pooling of this shape, materialise every head's proxy map in HBM and
+    keep each row's k largest blocks; returns the [B, H, N] selection as a bool
+    tensor view of the mask bits (see sol_attn_topk_route)."""
+    import torch
+    N = -(-L // BLOCK)
+    nw = -(-N // 32)
+    mask = torch.zeros(B, H, N, nw, device="cuda", dtype=torch.int32)
+    _check(lib().sol_attn_topk_route(B, H, L, d, BLOCK, int(k), mask.data_ptr(), _stream_handle(stream)))
+    return mask
 
 
 def workspace_bytes(B: int, H: int, L: int, d: int) -> int:

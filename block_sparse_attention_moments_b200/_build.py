@@ -10,7 +10,8 @@ ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libsol_attn.so")
 PROFILE_LIB = os.path.join(PKG, "libsol_attn_profile.so")
 SOURCES = [os.path.join(PKG, "csrc", "sol_attn.cu")]
-DEPS = [os.path.join(PKG, "csrc", f) for f in ("fused.cuh", "moments.cuh", "pool.cuh", "sm100_ptx.cuh")] + [
+DEPS = [os.path.join(PKG, "csrc", f) for f in ("fused.cuh", "moments.cuh", "pool.cuh", "sm100_ptx.cuh",
+                                                "topk_router.cuh")] + [
     os.path.join(ROOT, "include", "sol_attn.h")]
 
 NVCC_FLAGS = [

@@ -16,6 +16,7 @@
 #include "moments.cuh"
 #include "pool.cuh"
 #include "sol_attn.h"
+#include "topk_router.cuh"
 
 using namespace solattn;
 
@@ -72,6 +73,8 @@ struct Workspace {
   Shape last_fused;   // shape of the last completed forward (for stats)
   // host-buffer entry point: two staging slots, three streams (copy in,
   // compute, copy out) and the events that order them
+  void* topk_map = nullptr;   // proxy map of the comparison top-k router (grown on demand)
+  size_t topk_map_bytes = 0;
   void* host_stage = nullptr;
   size_t host_stage_bytes = 0;
   cudaStream_t host_stream = nullptr;   // copies in
@@ -613,6 +616,7 @@ int sol_attn_release(void) {
   if (w.base) CUDA_TRY(cudaFree(w.base));
   if (w.ctl_block) CUDA_TRY(cudaFree(w.ctl_block));
   if (w.host_stage) CUDA_TRY(cudaFree(w.host_stage));
+  if (w.topk_map) CUDA_TRY(cudaFree(w.topk_map));
   if (w.host_stream) CUDA_TRY(cudaStreamDestroy(w.host_stream));
   if (w.host_comp) CUDA_TRY(cudaStreamDestroy(w.host_comp));
   if (w.host_out) CUDA_TRY(cudaStreamDestroy(w.host_out));
@@ -717,6 +721,52 @@ int sol_attn_noalloc_status(void* stream) {
     return fail(SOL_ATTN_ERR_DEVICE, "device-side check failed: a tile descriptor was out of range (status 0x%x)",
                 h);
   }
+  return SOL_ATTN_OK;
+}
+
+int sol_attn_topk_route(int B, int H, int L, int d, int block, int k, uint32_t* mask, void* stream) {
+  int rc;
+  if ((rc = check_shape(B, H, L, d, block))) return rc;
+  if (!mask) return fail(SOL_ATTN_ERR_ARG, "mask is NULL");
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  Workspace& w = g_ws[dev];
+  if (!(w.shape == Shape{B, H, L, d}) || w.stage < 1)
+    return fail(SOL_ATTN_ERR_STATE, "topk_route needs a stage_pool or forward of the same shape first");
+  const int N = (L + kBlock - 1) / kBlock;
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t bytes = BH * N * N * sizeof(float);
+  if (w.topk_map_bytes < bytes) {
+    if (w.topk_map) CUDA_TRY(cudaFree(w.topk_map));
+    w.topk_map = nullptr;
+    w.topk_map_bytes = 0;
+    CUDA_TRY(cudaMalloc(&w.topk_map, bytes));
+    w.topk_map_bytes = bytes;
+  }
+  auto st = static_cast<cudaStream_t>(stream);
+  float* map = static_cast<float*>(w.topk_map);
+  const float isd = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  const dim3 grid((N + kMapTile - 1) / kMapTile, (N + kMapTile - 1) / kMapTile, static_cast<unsigned>(BH));
+  const size_t msm = 2u * kMapTile * (d + 1) * sizeof(float);
+  static bool attr_set[kMaxDevices] = {false};
+  if (!attr_set[dev]) {
+    CUDA_TRY(cudaFuncSetAttribute(proxy_map_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(2u * kMapTile * 129 * sizeof(float))));
+    CUDA_TRY(cudaFuncSetAttribute(proxy_map_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(2u * kMapTile * 65 * sizeof(float))));
+    CUDA_TRY(cudaFuncSetAttribute(topk_mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kMaxMaskWords * 32 * sizeof(uint32_t))));
+    attr_set[dev] = true;
+  }
+  if (d == 128)
+    proxy_map_kernel<128><<<grid, 256, msm, st>>>(w.qbar, w.kbar, N, isd, map);
+  else
+    proxy_map_kernel<64><<<grid, 256, msm, st>>>(w.qbar, w.kbar, N, isd, map);
+  CUDA_TRY(cudaGetLastError());
+  topk_mask_kernel<<<static_cast<unsigned>(BH * N), 256, static_cast<size_t>(N) * sizeof(uint32_t), st>>>(map, N, k,
+                                                                                                        mask);
+  CUDA_TRY(cudaGetLastError());
   return SOL_ATTN_OK;
 }
 

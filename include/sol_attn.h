@@ -178,6 +178,18 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
                              int B, int H, int L, int d, int block, int chunk, float beta,
                              void* stream);
 
+/* Comparison router for the routing-cost report (a measurement aid, not a step
+ * of the method; experiments: routing latency against top-k / top-p routers
+ * that materialise and traverse the proxy map, Fig. 5b/5c).  From the pooled
+ * Q̄, K̄ of the last sol_attn_stage_pool or forward of this shape on this
+ * device, writes the full proxy map ŝ_ij = Q̄_i·K̄_j/sqrt(d) of every head to
+ * HBM (fp32, B*H*N*N values, in a library-owned buffer grown with cudaMalloc)
+ * and keeps each row's k largest entries (ties: lower block index first) as
+ * bits of mask (device, [B,H,N,ceil(N/32)] uint32, caller-owned; k <= 0 keeps
+ * none, k >= N all).  Two kernels enqueued on stream.  SOL_ATTN_ERR_STATE
+ * without a matching earlier pooling. */
+int sol_attn_topk_route(int B, int H, int L, int d, int block, int k, uint32_t* mask, void* stream);
+
 /* Status of the last allocation-free forward on this device (the paper has no
  * counterpart).  That forward clears the device status word when it is
  * enqueued; this call synchronises stream, copies the word to the host (no

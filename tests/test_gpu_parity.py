@@ -334,3 +334,33 @@ def test_conflicting_flags_are_rejected():
     with pytest.raises(sa.SolAttnError) as e:
         sa.forward(q, k, v, 1.0, wl.chunk, flags=sa.FLAG_FIRST_ORDER | sa.FLAG_EXACT_ONLY)
     assert e.value.code == -1
+
+
+@pytest.mark.parametrize("kk", [0, 1, 13, 64])
+def test_topk_comparison_router(kk):
+    # The comparison router of the routing-cost report (experiments: top-k
+    # routing over the materialised proxy map, Fig. 5b): each row keeps exactly
+    # min(k, N) blocks, and every kept block's oracle proxy logit is at least
+    # every dropped one's (up to fp32 rounding of the map, 1e-4).
+    import torch
+    from oracle import pool_blocks, proxy_logits
+    from parity_util import to_device
+    from synth import bf16_bits_to_f64
+    wl = WORKLOADS["small"]
+    qb, kb, vb = fourier_inputs(wl)
+    q, k, v = to_device(qb), to_device(kb), to_device(vb)
+    sa.stage_pool(q, k, v)
+    mask = sa.topk_route(wl.B, wl.H, wl.L, wl.d, kk)
+    torch.cuda.synchronize()
+    w = mask.to(torch.int64).cpu().numpy() & 0xFFFFFFFF
+    N = wl.N
+    sel = ((w[..., :, None] >> np.arange(32)) & 1).reshape(wl.B, wl.H, N, -1)[..., :N].astype(bool)
+    for h in range(wl.H):
+        qbar, _, _ = pool_blocks(bf16_bits_to_f64(qb[0, h]))
+        kbar, _, _ = pool_blocks(bf16_bits_to_f64(kb[0, h]))
+        s = proxy_logits(qbar, kbar)
+        for i in range(N):
+            row = sel[0, h, i]
+            assert row.sum() == min(kk, N)
+            if 0 < kk < N:
+                assert s[i][row].min() >= s[i][~row].max() - 1e-4
