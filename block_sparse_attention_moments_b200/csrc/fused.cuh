@@ -40,7 +40,8 @@
 //   warp 10    routing: fetches the next item, computes ŝ_ij = Q̄_i·K̄_j/sqrt(d)
 //              in fp32 for both halves, compares with τ_i (warp ballot -> mask
 //              words), one item ahead (double-buffered mask slots).
-//   warp 11    scheduler: walks each item's tile sequence from its masks and
+//   warp 11    scheduler: walks each item's tile sequence from its masks (the
+//              union blocks of a chunk listed by all 32 lanes at once) and
 //              publishes one descriptor per tile (blocks, column validity per
 //              half, first/last flags) into a shared-memory ring that the
 //              producers, both MMA issuers and the softmax warps consume.
@@ -64,7 +65,7 @@
 // so the only shared-memory operand traffic is Q, K and V.
 //
 // Shared memory (1024-byte aligned, 128-byte swizzled tiles):
-//   Q 32 KB | K ring 2 x 32 KB | V ring 2 x 32 KB | control.
+//   Q 32 KB | K ring 2 x 32 KB | V ring 3 x 32 KB | control.
 // TMEM (512 columns): O [0,128), S/P buffers b = t mod 3 at [128 + 128 b, 256 + 128 b).
 #pragma once
 
@@ -125,6 +126,7 @@ struct FusedParams {
 };
 
 constexpr int kStages = 2;
+constexpr int kStagesV = 3;   // V ring: a stage is free once the PV of its tile completed
 
 // One entry of the tile sequence, published by the scheduler warp.
 struct __align__(16) TileDesc {
@@ -142,6 +144,9 @@ constexpr int kDescApprox = 4;   // approximation tile (else exact)
 constexpr int kDescEmpty = 8;    // item without any tile (exact-only, nothing selected)
 constexpr int kDescEnd = 16;     // no more work
 constexpr int kRing = 8;         // descriptor ring entries
+constexpr int kListPass = 1024;                 // blocks examined per listing pass
+constexpr int kListCap = kListPass + 32;        // listed blocks held (a pass plus a leftover)
+
 
 struct __align__(16) ItemSlot {
   uint32_t mask[2][kMaxMaskWords];  // selection bits of both halves
@@ -154,13 +159,14 @@ struct __align__(16) FusedCtl {
   ItemSlot slot[2];
   TileDesc ring[kRing];             // scheduler -> producers, MMA issuers, softmax
   float qbar[2][128];               // routing: pooled queries of the pair
+  uint16_t ulist[kListCap];         // scheduler: union blocks of the current chunk in walk order
   float hand[3][128];               // [tile % 3][row]: the m tile t settled on, read by tile t + 1
   float2 xval[2][2][128];           // epilogue: [parity][warpgroup][row] partial (row sum, its m)
   uint64_t item_full[2], item_empty[2];
   uint64_t ring_full[kRing], ring_empty[kRing];
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages];         // K-side stage loaded (its reuse waits for the S MMA: s_full)
-  uint64_t v_full[kStages];         // V-side stage loaded (its reuse waits for the PV MMA: pv_done)
+  uint64_t v_full[kStagesV];        // V-side stage loaded (its reuse waits for the PV MMA: pv_done)
   uint64_t s_full[3], p_full[3];    // per TMEM S buffer (tile index % 3)
   uint64_t pv_done[3];              // per TMEM S buffer: its PV completed
   uint64_t mready[3];               // per TMEM S buffer: hand[] of that tile written
@@ -175,7 +181,7 @@ constexpr uint32_t kTile = 32768;  // 128 rows x 128 bf16
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + kTile;
 constexpr uint32_t kSmemV = kSmemK + kStages * kTile;
-constexpr uint32_t kSmemCtl = kSmemV + kStages * kTile;
+constexpr uint32_t kSmemCtl = kSmemV + kStagesV * kTile;
 constexpr uint32_t kFusedSmemBytes = kSmemCtl + sizeof(FusedCtl) + 1024;  // + alignment slack
 static_assert(kFusedSmemBytes <= 227u * 1024u, "dynamic shared memory of one CTA on sm_100");
 constexpr uint32_t kTmemCols = 512;
@@ -213,60 +219,84 @@ struct Tile {
 // chunk at block i0, then wraps around.  The online softmax is independent of
 // the order of its tiles up to rounding; starting near the diagonal makes the
 // first tiles carry each row's largest logits, so the running maximum rarely
-// moves afterwards.  Run by the scheduler warp.
+// moves afterwards.  Run by the whole scheduler warp (warp-collective): the
+// union blocks of a chunk are listed 1024 at a time, each lane taking 32
+// blocks, with a warp prefix sum of their counts placing them in order.
 struct TileIter {
   const uint32_t* m0;
   const uint32_t* m1;
+  uint16_t* list;   // shared memory, kListCap entries
   int N, C, W;
   int nw;           // mask words per half
   bool has1, exact_only, first;
   bool all_blocks;  // walk every block as exact (first-order mode), whatever the selection
   int lo, hi;       // current chunk [lo, hi)
   int jstart;       // the chunk's exact blocks run over [jstart, hi) then [lo, jstart)
-  int seg;          // 0, 1: position in those two ranges; 2: exact blocks done
-  int j;            // next candidate block of the current range
+  int seg;          // 0, 1: position in those two ranges; 2: exact blocks listed
+  int scan;         // next block of the current range not yet listed
+  int n, k;         // blocks listed, next one to emit
   int a0;           // next approximation sub-tile start
   int chunks_left;
 
-  // First block of the union of both selections in [from, lim), or lim.
-  __device__ __forceinline__ int next_union(int from, int lim) const {
-    int x = from;
-    while (x < lim) {
-      const int w = x >> 5;
-      const uint32_t u = (all_blocks ? 0xFFFFFFFFu : (m0[w] | m1[w])) & (0xFFFFFFFFu << (x & 31));
-      if (u) {
-        const int jj = (w << 5) + __ffs(u) - 1;
-        return jj < lim ? jj : lim;
-      }
-      x = (w + 1) << 5;
+  // Lists further union blocks in walk order until at least two wait to be
+  // emitted or the chunk's ranges are exhausted.
+  __device__ __forceinline__ void refill(int lane) {
+    if (k > 0) {   // keep a leftover block at the front
+      const int keep = n - k;
+      const uint16_t v = (keep > 0) ? list[k] : 0;
+      __syncwarp();
+      if (keep > 0 && lane == 0) list[0] = v;
+      __syncwarp();
+      n = keep;
+      k = 0;
     }
-    return lim;
-  }
-  // Next selected block of the current chunk in its exact order, or -1.
-  __device__ __forceinline__ int next_exact() {
-    while (seg < 2) {
+    while (seg < 2 && n < 2) {
       const int lim = seg == 0 ? hi : jstart;
-      const int jj = next_union(j, lim);
-      if (jj < lim) {
-        j = jj + 1;
-        return jj;
+      if (scan >= lim) {
+        ++seg;
+        scan = lo;
+        continue;
       }
-      ++seg;
-      j = lo;
+      const int wb = scan + 32 * lane;
+      uint32_t u = 0u;
+      if (wb < lim) {
+        u = all_blocks ? 0xFFFFFFFFu : (mask_bits32(m0, wb, nw) | mask_bits32(m1, wb, nw));
+        const int nv = lim - wb;
+        if (nv < 32) u &= (1u << nv) - 1u;
+      }
+      const int c = __popc(u);
+      int pre = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+        if (lane >= o) pre += v;
+      }
+      const int tot = __shfl_sync(0xFFFFFFFFu, pre, 31);
+      int pos = n + pre - c;
+      while (u) {
+        const int bb = __ffs(u) - 1;
+        u &= u - 1u;
+        list[pos++] = static_cast<uint16_t>(wb + bb);
+      }
+      __syncwarp();
+      n += tot;
+      scan = min(scan + kListPass, lim);
     }
-    return -1;
   }
   __device__ __forceinline__ void start_chunk(int start) {
     hi = min(lo + C, N);
     jstart = start;
     seg = 0;
-    j = start;
+    scan = start;
+    n = 0;
+    k = 0;
     a0 = exact_only ? hi : lo;
   }
-  __device__ __forceinline__ void init(const ItemSlot& s, int N_, int C_, int W_, int i0, bool has1_,
-                                       bool exact_only_) {
+  __device__ __forceinline__ void init(const ItemSlot& s, uint16_t* list_, int N_, int C_, int W_, int i0,
+                                       bool has1_, bool exact_only_) {
     m0 = s.mask[0];
     m1 = s.mask[1];
+    list = list_;
     N = N_;
     C = C_;
     W = W_;
@@ -279,11 +309,13 @@ struct TileIter {
     lo = (i0 / C_) * C_;
     start_chunk(i0);
   }
-  __device__ __forceinline__ bool next(Tile& t) {
+  __device__ __forceinline__ bool next(Tile& t, int lane) {
     while (chunks_left > 0) {
-      const int ja = next_exact();
-      if (ja >= 0) {
-        const int jb = next_exact();
+      if (n - k < 2 && seg < 2) refill(lane);
+      if (k < n) {
+        const int ja = list[k];
+        const int jb = (k + 1 < n) ? static_cast<int>(list[k + 1]) : -1;
+        k += (jb >= 0) ? 2 : 1;
         t = (jb >= 0) ? Tile{1, ja, jb, 128, 0, first} : Tile{1, ja, -1, 64, 0, first};
         first = false;
         return true;
@@ -294,8 +326,8 @@ struct TileIter {
         a0 = a1;
         bool any = false;
         for (int x = s; x < a1 && !any; x += 32) {
-          const int n = min(32, a1 - x);
-          const uint32_t range = (n >= 32) ? 0xFFFFFFFFu : ((1u << n) - 1u);
+          const int nn = min(32, a1 - x);
+          const uint32_t range = (nn >= 32) ? 0xFFFFFFFFu : ((1u << nn) - 1u);
           uint32_t unsel = ~mask_bits32(m0, x, nw);
           if (has1) unsel |= ~mask_bits32(m1, x, nw);
           any = (unsel & range) != 0u;
@@ -365,6 +397,43 @@ __device__ __forceinline__ float exp2_neg_int(float k) {
   return (ki >= 126) ? 0.f : __int_as_float((127 - ki) << 23);
 }
 
+// Out-of-line pieces of the softmax path that run rarely (once per item, or on
+// a rescale), so that the per-tile code stays small.
+// The row's O (its first d columns) times alpha, a power of two.  Warp-wide.
+__device__ __noinline__ void scale_o(uint32_t tO, float alpha, int d) {
+#pragma unroll 1
+  for (int c = 0; c < d; c += 32) {
+    float o[32];
+    tmem_ld_x32f(tO + c, o);
+    tmem_ld_wait();
+    reg_fence32(o);
+    uint32_t ow[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ow[e] = __float_as_uint(o[e] * alpha);
+    tmem_st_x32(tO + c, ow);
+  }
+}
+__device__ __noinline__ void store_o_rows(uint32_t tO, int c_lo, int c_hi, bool have, float inv_l, uint16_t* orow) {
+#pragma unroll 1
+  for (int c16 = c_lo; c16 < c_hi; c16 += 16) {
+    float a[16];
+    if (have) {
+      tmem_ld_x16f(tO + c16, a);
+      tmem_ld_wait();
+      reg_fence16(a);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) a[e] = 0.f;
+    }
+    if (orow) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c16);
+      dst[0] = make_uint4(pack_bf16x2(a[0] * inv_l, a[1] * inv_l), pack_bf16x2(a[2] * inv_l, a[3] * inv_l),
+                          pack_bf16x2(a[4] * inv_l, a[5] * inv_l), pack_bf16x2(a[6] * inv_l, a[7] * inv_l));
+      dst[1] = make_uint4(pack_bf16x2(a[8] * inv_l, a[9] * inv_l), pack_bf16x2(a[10] * inv_l, a[11] * inv_l),
+                          pack_bf16x2(a[12] * inv_l, a[13] * inv_l), pack_bf16x2(a[14] * inv_l, a[15] * inv_l));
+    }
+  }
+}
 // FO: the first-order mode (kFlagFirstOrder) is a separate instantiation, so
 // that its extra per-tile work does not enter the default kernel's code.
 template <int D, bool FO>
@@ -405,10 +474,8 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
       mbar_init(&ctl.ring_full[r], 1);
       mbar_init(&ctl.ring_empty[r], kRingEmptyCount);
     }
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ctl.k_full[s], 1);
-      mbar_init(&ctl.v_full[s], 1);
-    }
+    for (int s = 0; s < kStages; ++s) mbar_init(&ctl.k_full[s], 1);
+    for (int s = 0; s < kStagesV; ++s) mbar_init(&ctl.v_full[s], 1);
     mbar_init(&ctl.q_full, 1);
     mbar_init(&ctl.q_empty, 1);
     mbar_init(&ctl.xchg, 8);   // one arrival per softmax warp
@@ -575,14 +642,14 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
         publish();
       } else {
         TileIter it;
-        it.init(sl, p.N, p.chunk, p.W, 2 * pair, 2 * pair + 1 < p.N, exact_only || first_order);
+        it.init(sl, ctl.ulist, p.N, p.chunk, p.W, 2 * pair, 2 * pair + 1 < p.N, exact_only || first_order);
         it.all_blocks = first_order;
         Tile t, tn;
-        bool have = it.next(t);
+        bool have = it.next(t, lane);
         bool first_desc = true;
         while (have) {
           SA_PROF(const unsigned long long tn0 = clock64();)
-          const bool have_next = it.next(tn);
+          const bool have_next = it.next(tn, lane);
           SA_PROF(prof[kPrSchedNext] += clock64() - tn0;)
           if (!first_desc && !(dsc = claim())) break;
           first_desc = false;
@@ -661,12 +728,14 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
             tma_load_3d(sQ + cb * CB, &tm_q, &ctl.q_full, cb * 64, 128 * pair, bh);
           ++qseq;
         }
-        // The stage was last used by tile tl - kStages; it is free once that
-        // tile's S MMA (K side) or PV MMA (V side) has completed, which the
-        // barriers of its TMEM buffer (tl - kStages) % 3 record.
+        // The stage was last used by tile tl - nst (nst stages on this side);
+        // it is free once that tile's S MMA (K side) or PV MMA (V side) has
+        // completed, which the barriers of its TMEM buffer (tl - nst) % 3
+        // record.
         uint64_t* full = kside ? &ctl.k_full[stage] : &ctl.v_full[stage];
-        if (tl >= kStages) {
-          const uint32_t tp = tl - kStages;
+        const uint32_t nst = kside ? kStages : kStagesV;
+        if (tl >= nst) {
+          const uint32_t tp = tl - nst;
           uint64_t* done = kside ? &ctl.s_full[tp % 3u] : &ctl.pv_done[tp % 3u];
           if (!wait(done, (tp / 3u) & 1u, kside ? kPrKEmpty : kPrVEmpty)) break;
         }
@@ -693,7 +762,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
             if (nblk == 2) tma_load_3d(dst + cb * CB + 8192, map, full, cb * 64, 64 * jb, bh);
           }
         }
-        if (++stage == kStages) stage = 0;
+        if (++stage == static_cast<int>(nst)) stage = 0;
       }
     }
   } else {
@@ -790,7 +859,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
         }
         umma_commit(&ctl.pv_done[b]);
         SA_PROF(prof[kPrPvIssue] += clock64() - tis;)
-        if (++vstage == kStages) {
+        if (++vstage == kStagesV) {
           vstage = 0;
           vphase ^= 1u;
         }
@@ -977,17 +1046,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
             if (!wait_w(&ctl.pv_done[(t - 1u) % 3u], ((t - 1u) / 3u) & 1u, kPrSmO)) break;
             tc_fence_after();
             const float alpha = o_behind ? exp2_neg_int(m_fin - m_hand) : 1.f;
-#pragma unroll 1
-            for (int c = 0; c < D; c += 32) {
-              float o[32];
-              tmem_ld_x32f(tO + c, o);
-              tmem_ld_wait();
-              reg_fence32(o);
-              uint32_t ow[32];
-#pragma unroll
-              for (int e = 0; e < 32; ++e) ow[e] = __float_as_uint(o[e] * alpha);
-              tmem_st_x32(tO + c, ow);
-            }
+            scale_o(tO, alpha, D);
             SA_PROF(prof[kPrSmRescales] += 1;)
           }
           ctl.hand[b][row] = m_fin;
@@ -1033,25 +1092,7 @@ __global__ void __launch_bounds__(kLaunchBoundThreads, 1)
       const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
       const int token = 128 * dpair + row;
       uint16_t* orow = p.out + (static_cast<size_t>(dbh) * p.L + token) * D;
-#pragma unroll 1
-      for (int c16 = wg * (D / 2); c16 < (wg + 1) * (D / 2); c16 += 16) {
-        float a[16];
-        if (item_tiles) {
-          tmem_ld_x16f(tO + c16, a);
-          tmem_ld_wait();
-          reg_fence16(a);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) a[e] = 0.f;
-        }
-        if (token < p.L) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c16);
-          dst[0] = make_uint4(pack_bf16x2(a[0] * inv_l, a[1] * inv_l), pack_bf16x2(a[2] * inv_l, a[3] * inv_l),
-                              pack_bf16x2(a[4] * inv_l, a[5] * inv_l), pack_bf16x2(a[6] * inv_l, a[7] * inv_l));
-          dst[1] = make_uint4(pack_bf16x2(a[8] * inv_l, a[9] * inv_l), pack_bf16x2(a[10] * inv_l, a[11] * inv_l),
-                              pack_bf16x2(a[12] * inv_l, a[13] * inv_l), pack_bf16x2(a[14] * inv_l, a[15] * inv_l));
-        }
-      }
+      store_o_rows(tO, wg * (D / 2), (wg + 1) * (D / 2), item_tiles, inv_l, token < p.L ? orow : nullptr);
       // O is read; the next item's first PV (which overwrites O) waits for this
       // warp's arrival on that tile, which comes after these reads
       tc_fence_before();
