@@ -98,6 +98,20 @@ def test_chunk_size_does_not_change_the_result():
         assert np.abs(out - ref_out).max() <= 2e-2
 
 
+@pytest.mark.parametrize("chunk", [1100, 4096])
+def test_window_wider_than_one_listing_pass(chunk):
+    # The tile walk lists a window's union blocks 1024 at a time; a window of
+    # C > 1024 pooled keys (N = 2304 here, so C = 4096 puts every block in one
+    # window) needs several passes and a block carried between them.
+    qb, kb, vb = custom_fourier(1, 2, (9, 64, 256), 128, 3.0, seed=91)
+    N = qb.shape[2] // 64
+    rows = [0, 1, 700, 1151, 1152, N - 2, N - 1]
+    ref_out, ref_sel, _ = _full_check(qb, kb, vb, 1.0, 64, rows=rows)
+    out, sel, _ = _full_check(qb, kb, vb, 1.0, chunk, rows=rows, mask_heads=[1])
+    assert (sel == ref_sel).all()
+    assert np.abs(out - ref_out).max() <= 2e-2
+
+
 def test_select_all_flag_equals_dense_beta():
     wl = WORKLOADS["small"]
     qb, kb, vb = fourier_inputs(wl)
